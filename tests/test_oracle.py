@@ -1,0 +1,268 @@
+"""Pins of the CPU oracle against things other than itself: hand-derived
+golden examples, closed forms, library reductions (torch softmax, a dense
+SwiGLU MLP written with torch.nn.functional), dense-mask brute force,
+invariants and exact special cases. CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+BF16 = torch.bfloat16
+
+
+def bf16(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(BF16)
+
+
+# ---------------------------------------------------------------- rounding
+def test_round_bf16_matches_torch_on_float32_values():
+    g = torch.Generator().manual_seed(0)
+    v = torch.randn(200000, generator=g) * torch.exp(torch.randn(200000, generator=g) * 20)
+    v = torch.cat([v, torch.tensor([0.0, -0.0, 1e-40, -3e-39, 3.3e38, -3.39e38, float("inf"), float("-inf")])])
+    ours = oracle.round_bf16(v.double())
+    ref = v.to(BF16)  # float32 -> bf16 is a single RNE rounding in torch
+    assert torch.equal(ours.view(torch.int16), ref.view(torch.int16))
+
+
+def test_round_bf16_ties_and_single_rounding():
+    cases = {
+        1 + 2.0 ** -8: 1.0,  # halfway, ties to even (down)
+        1 + 3 * 2.0 ** -8: 1 + 2.0 ** -6,  # halfway, ties to even (up)
+        1 + 2.0 ** -8 + 2.0 ** -40: 1 + 2.0 ** -7,  # just above halfway: a float first step would lose this
+        -(1 + 2.0 ** -8 + 2.0 ** -40): -(1 + 2.0 ** -7),
+        2.0 ** -133: 2.0 ** -133,  # smallest bf16 subnormal
+        2.0 ** -134: 0.0,  # halfway to the smallest subnormal -> even (0)
+    }
+    inp = torch.tensor(list(cases.keys()), dtype=torch.float64)
+    out = oracle.round_bf16(inp).double()
+    assert out.tolist() == list(cases.values())
+
+
+# ---------------------------------------------------------------- golden
+def _golden_inputs(ex):
+    x, Wr, br = bf16(ex["x"]), bf16(ex["Wr"]), bf16(ex["br"])
+    W1, b1, W2, b2 = bf16(ex["W1"]), bf16(ex["b1"]), bf16(ex["W2"]), bf16(ex["b2"])
+    return x, Wr, br, W1, b1, W2, b2
+
+
+@pytest.mark.parametrize("name", ["top1_swiglu", "top2_softmax", "tie_lower_index"])
+def test_golden_worked_examples(name):
+    data = json.load(open(os.path.join(GOLDEN, "worked_examples.json")))
+    ex = next(e for e in data["examples"] if e["name"] == name)
+    x, Wr, br, W1, b1, W2, b2 = _golden_inputs(ex)
+    y, idx, w = oracle.forward(x, Wr, br, W1, b1, W2, b2, ex["k"])
+    assert idx.tolist() == ex["topk_idx"]
+    np.testing.assert_allclose(w.numpy(), np.asarray(ex["topk_w"]), rtol=1e-7, atol=0)
+    assert y.float().tolist() == ex["y"]
+
+
+def test_e2m1_table():
+    data = json.load(open(os.path.join(GOLDEN, "e2m1_table.json")))
+    for s_str, scale in data["scales"].items():
+        s = int(s_str)
+        codes = torch.tensor([[c | (c << 4) for c in range(0, 16, 1)] * 2], dtype=torch.uint8)  # 32 bytes = 64 values
+        codes = codes[:, :32]
+        scales = torch.full((1, 2), s, dtype=torch.uint8)
+        vals = oracle.dequant_mxfp4(codes, scales)[0]
+        for i in range(64):
+            code = i // 2 % 16
+            expect = data["codes"][str(code)] * scale
+            assert vals[i].item() == expect, (s, i, code)
+            if code == 8:
+                assert math.copysign(1.0, vals[i].item()) == -1.0
+
+
+# ---------------------------------------------------------------- router
+def _rank_mask(logits64_f32, k):
+    """Dense brute force: expert e is chosen iff fewer than k experts beat it
+    under (logit desc, index asc)."""
+    L = logits64_f32
+    T, E = L.shape
+    mask = np.zeros((T, E), dtype=bool)
+    rank = np.zeros((T, E), dtype=np.int64)
+    for e in range(E):
+        beats = (L > L[:, e:e + 1]) | ((L == L[:, e:e + 1]) & (np.arange(E)[None, :] < e))
+        rank[:, e] = beats.sum(axis=1)
+    mask = rank < k
+    return mask, rank
+
+
+@pytest.mark.parametrize("T,D,E,k", [(37, 48, 6, 2), (16, 64, 4, 4), (50, 32, 16, 5), (9, 8, 3, 1)])
+def test_route_matches_dense_mask_brute_force(T, D, E, k):
+    inp = synthetic.make_custom(T, D, E, k, 8, seed=T + D)
+    logits, idx, w = oracle.route(inp.x, inp.Wr, inp.br, k)
+    L = inp.x.double().numpy() @ inp.Wr.double().numpy().T + inp.br.double().numpy()[None, :]
+    np.testing.assert_allclose(logits.numpy(), L, rtol=1e-6, atol=1e-6)
+    Lf = logits.numpy().astype(np.float64)
+    mask, rank = _rank_mask(Lf, k)
+    # softmax restricted to the chosen experts (others get -inf)
+    masked = np.where(mask, Lf, -np.inf)
+    p = np.exp(masked - masked.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    for t in range(T):
+        chosen = sorted(np.nonzero(mask[t])[0], key=lambda e: rank[t, e])
+        assert idx[t].tolist() == chosen
+        np.testing.assert_allclose(w[t].numpy(), p[t, chosen], rtol=2e-7, atol=1e-9)
+
+
+def test_route_k_equals_E_is_plain_softmax():
+    inp = synthetic.make_custom(64, 32, 8, 8, 8, seed=3)
+    logits, idx, w = oracle.route(inp.x, inp.Wr, inp.br, 8)
+    ref = torch.softmax(logits.double(), dim=1)
+    for t in range(64):
+        np.testing.assert_allclose(w[t].numpy(), ref[t, idx[t].long()].numpy(), rtol=2e-7)
+        assert sorted(idx[t].tolist()) == list(range(8))
+
+
+def test_route_exact_ties_pick_lower_index():
+    # integer-valued inputs; duplicated router rows make exact ties
+    T, D, E, k = 12, 4, 6, 3
+    g = torch.Generator().manual_seed(5)
+    x = torch.randint(-3, 4, (T, D), generator=g).to(BF16)
+    base = torch.randint(-2, 3, (3, D), generator=g)
+    Wr = torch.cat([base, base]).to(BF16)  # expert e and e+3 share weights
+    br = torch.zeros(E, dtype=BF16)
+    logits, idx, w = oracle.route(x, Wr, br, k)
+    L = logits.double().numpy()
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-L[t, e], e))[:k]
+        assert idx[t].tolist() == order
+        for j in range(k - 1):
+            if L[t, idx[t, j]] == L[t, idx[t, j + 1]]:
+                assert idx[t, j] < idx[t, j + 1]
+                assert w[t, j] == w[t, j + 1]
+
+
+def test_route_invariants():
+    inp = synthetic.make_inputs("debug", T=512)
+    logits, idx, w = oracle.route(inp.x, inp.Wr, inp.br, 2)
+    assert torch.all((idx >= 0) & (idx < 8))
+    assert all(len(set(r)) == 2 for r in idx.tolist())
+    np.testing.assert_allclose(w.double().sum(1).numpy(), 1.0, atol=1e-6)
+    assert torch.all(w[:, 0] >= w[:, 1])
+    # the chosen logits are the two largest
+    top = torch.topk(logits, 2, dim=1).values
+    assert torch.equal(torch.gather(logits, 1, idx.long()), top)
+
+
+# ---------------------------------------------------------------- permutation
+@pytest.mark.parametrize("T,E,k", [(100, 7, 3), (1, 4, 4), (257, 16, 2), (64, 128, 4)])
+def test_permute_is_stable_sort_by_expert(T, E, k):
+    g = torch.Generator().manual_seed(T * E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    counts, offsets, perm, inv = oracle.permute(idx, E)
+    flat = idx.flatten().numpy()
+    ref_perm = np.argsort(flat, kind="stable")
+    assert perm.numpy().tolist() == ref_perm.tolist()
+    assert counts.numpy().tolist() == np.bincount(flat, minlength=E).tolist()
+    assert offsets.numpy().tolist() == [0] + np.cumsum(np.bincount(flat, minlength=E)).tolist()
+    assert int(counts.sum()) == T * k
+    assert torch.equal(inv[perm.long()], torch.arange(T * k, dtype=torch.int32))
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]].numpy()
+        assert np.all(np.diff(seg) > 0)
+        assert np.all(flat[seg] == e)
+
+
+def test_permute_rejects_out_of_range_index():
+    idx = torch.tensor([[0, 5]], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        oracle.permute(idx, 4)
+
+
+# ---------------------------------------------------------------- expert FFN
+def _dense_swiglu_reference(x, W1, b1, W2, b2, I):
+    """A dense SwiGLU MLP with torch.nn.functional (float64), h rounded to bf16."""
+    u = F.linear(x.double(), W1.double(), b1.double())
+    h = (F.silu(u[:, :I]) * u[:, I:]).float().to(BF16).double()
+    return F.linear(h, W2.double(), b2.double())
+
+
+def test_ffn_single_expert_is_dense_swiglu_mlp():
+    T, D, I = 24, 64, 48
+    inp = synthetic.make_custom(T, D, 1, 1, I, seed=11)
+    y, idx, w = oracle.forward(inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, 1)
+    assert torch.all(idx == 0) and torch.all(w == 1.0)
+    ref = _dense_swiglu_reference(inp.x, inp.W1[0], inp.b1[0], inp.W2[0], inp.b2[0], I)
+    # one bf16 rounding of y (and h rounding through float here) -> within 2 bf16 ulps
+    np.testing.assert_allclose(y.double().numpy(), ref.numpy(), rtol=2 ** -7, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,D,E,k,I", [(20, 32, 5, 2, 16), (8, 64, 3, 3, 32)])
+def test_ffn_matches_dense_all_expert_brute_force(T, D, E, k, I):
+    inp = synthetic.make_custom(T, D, E, k, I, seed=7 * T + E, reject=oracle.gap_reject())
+    y, o = None, None
+    logits, idx, w = oracle.route(inp.x, inp.Wr, inp.br, k)
+    y, o = oracle.ffn_tokens(inp.x, idx, w, inp.W1, inp.b1, inp.W2, inp.b2, return_o=True)
+    # brute force: every expert on every token, then a dense gate mask
+    mask, rank = _rank_mask(logits.double().numpy(), k)
+    gate = np.zeros((T, E))
+    for t in range(T):
+        for j in range(k):
+            gate[t, idx[t, j]] = w[t, j].item()
+    assert np.all((gate > 0) == mask)
+    y_dense = np.zeros((T, D))
+    for e in range(E):
+        o_e = _dense_swiglu_reference(inp.x, inp.W1[e], inp.b1[e], inp.W2[e], inp.b2[e], I).numpy()
+        y_dense += gate[:, e:e + 1] * o_e
+        for t in range(T):
+            for j in range(k):
+                if idx[t, j] == e:
+                    np.testing.assert_allclose(o[t, j].numpy(), o_e[t], rtol=1e-2, atol=1e-5)
+    np.testing.assert_allclose(y.double().numpy(), y_dense, rtol=2 ** -7, atol=1e-5)
+
+
+def test_w2_zero_gives_weighted_bias_sum():
+    T, D, E, k, I = 16, 32, 6, 3, 16
+    inp = synthetic.make_custom(T, D, E, k, I, seed=2)
+    W2 = torch.zeros_like(inp.W2)
+    y, idx, w = oracle.forward(inp.x, inp.Wr, inp.br, inp.W1, inp.b1, W2, inp.b2, k)
+    ref = (w.double()[:, :, None] * inp.b2.double()[idx.long()]).sum(1)
+    assert torch.equal(y, oracle.round_bf16(ref))
+
+
+def test_equivariance_under_token_and_expert_relabelling():
+    T, D, E, k, I = 24, 32, 6, 2, 16
+    inp = synthetic.make_custom(T, D, E, k, I, seed=9, reject=oracle.gap_reject())
+    y, idx, w = oracle.forward(inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, k)
+    pt = torch.randperm(T, generator=torch.Generator().manual_seed(1))
+    y2, _, _ = oracle.forward(inp.x[pt], inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, k)
+    assert torch.equal(y2, y[pt])
+    pe = torch.randperm(E, generator=torch.Generator().manual_seed(2))
+    y3, idx3, _ = oracle.forward(inp.x, inp.Wr[pe], inp.br[pe], inp.W1[pe], inp.b1[pe], inp.W2[pe], inp.b2[pe], k)
+    assert torch.equal(y3, y)
+    assert torch.equal(pe[idx3.long()].int(), idx)
+
+
+# ---------------------------------------------------------------- MXFP4
+def test_mxfp4_layer_equals_bf16_layer_with_dequantized_weights():
+    T, D, E, k, I = 16, 64, 4, 2, 64
+    inp = synthetic.make_custom(T, D, E, k, I, seed=4, wfmt="mxfp4")
+    y4, idx4, w4 = oracle.forward(inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, k,
+                                  W1_scales=inp.W1_scales, W2_scales=inp.W2_scales)
+    W1d = torch.stack([oracle.dequant_mxfp4(inp.W1[e], inp.W1_scales[e]) for e in range(E)])
+    W2d = torch.stack([oracle.dequant_mxfp4(inp.W2[e], inp.W2_scales[e]) for e in range(E)])
+    W1b, W2b = W1d.to(BF16), W2d.to(BF16)
+    assert torch.equal(W1b.double(), W1d) and torch.equal(W2b.double(), W2d)  # exact in bf16
+    yb, idxb, wb = oracle.forward(inp.x, inp.Wr, inp.br, W1b, inp.b1, W2b, inp.b2, k)
+    assert torch.equal(idx4, idxb)
+    assert torch.equal(y4.view(torch.int16), yb.view(torch.int16))
+
+
+def test_mxfp4_nibble_order_and_scale_blocks():
+    # one row, K=64: element 2m is the low nibble of byte m; scale block b covers 32b..32b+31
+    codes = torch.zeros((1, 32), dtype=torch.uint8)
+    codes[0, 0] = 0x72  # element 0 -> code 2 (1.0), element 1 -> code 7 (6.0)
+    codes[0, 16] = 0x0b  # element 32 -> code 11 (-1.5)
+    scales = torch.tensor([[127, 125]], dtype=torch.uint8)
+    v = oracle.dequant_mxfp4(codes, scales)[0]
+    assert v[0].item() == 1.0 and v[1].item() == 6.0 and v[32].item() == -1.5 * 0.25
+    assert torch.count_nonzero(v).item() == 3
