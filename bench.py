@@ -1,0 +1,360 @@
+"""Benchmark of the GPT-OSS-style MoE feed-forward layer on B200.
+
+One step = one pass of the whole layer (route, permute, gather, mlp1, mlp2,
+combine) over one batch of the GPT-OSS-20B-shaped workload (T=8192 tokens,
+D=2880, E=32 experts, top-4, I=2880, bf16, synthetic seeded inputs), timed on
+the device with CUDA events on the launching stream. Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU under torchrun; tokens are independent, so each
+rank runs its own batch with replicated weights and no collective on the data
+path (weak scaling); the step time is the max over ranks.
+``--impl reference`` times the CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+WORKLOAD = "gptoss20b"
+METRIC = "MoE layer tokens/s and TFLOP/s at 1 B200, % of tensor-core peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels per step: route 1, permute 2, gather 1, mlp1 1, mlp2 1, combine 1
+LAUNCHES_PER_STEP = 7
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        smax = float(rows[0][2])
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]"))}
+
+
+def traffic_from_profile(kernel_src: str):
+    """DRAM bytes per launch of the mlp1 kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "mlp1_gptoss20b_ncu.md")
+    if not os.path.exists(p):
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    fields = {}
+    for line in open(p):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256_16") != sha:
+        return None
+    try:
+        return int(float(fields["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import mixture_experts_ffn_layer_b200 as moe
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    shape = synthetic.SHAPES[WORKLOAD]
+    inp = synthetic.make_inputs(WORKLOAD, seed=synthetic.SEEDS[WORKLOAD] + 1000 * rank, device=dev)
+    T, D, E, k, I = shape.T, shape.D, shape.E, shape.k, shape.I
+    R = T * k
+    d = moe.dims(T, D, E, k, I)
+    ws = moe.alloc_workspace(d, device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    topk_idx = torch.empty((T, k), **i32)
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    perm, inv = torch.empty(R, **i32), torch.empty(R, **i32)
+    x_perm = torch.empty((R, D), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((R, I), dtype=torch.bfloat16, device=dev)
+    o_perm = torch.empty((R, D), dtype=torch.float32, device=dev)
+    y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    stages = ["route", "permute", "gather", "mlp1", "mlp2", "combine"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+
+        mark(0)
+        moe.moe_route(d, inp.x, inp.Wr, inp.br, topk_idx, topk_w)
+        mark(1)
+        moe.moe_permute(d, topk_idx, counts, offsets, perm, inv, ws)
+        mark(2)
+        moe.moe_gather(d, inp.x, perm, x_perm, ws)
+        mark(3)
+        moe.moe_mlp1(d, x_perm, offsets, inp.W1, inp.b1, h, ws)
+        mark(4)
+        moe.moe_mlp2(d, h, perm, offsets, topk_w, inp.W2, inp.b2, o_perm, ws)
+        mark(5)
+        moe.moe_combine(d, o_perm, inv, y, ws)
+        mark(6)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    st = moe.moe_read_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.status_str(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier()
+    with Clocks(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    st = moe.moe_read_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {moe.status_str(st)}")
+    stage_ms = {s: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i, s in enumerate(stages)}
+
+    # end to end through the one-call API with host buffers: H2D of x, forward, D2H of y
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_forward(d, x_dev, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([elapsed_ms, e2e_ms, stage_ms["mlp1"]], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, mlp1_ms = times.tolist()
+    ms_per_step = elapsed_ms / args.steps
+    tokens_total = T * world
+    value = tokens_total / (ms_per_step / 1e3)
+    tflops = shape.flops * world / (ms_per_step / 1e3) / 1e12
+
+    pk, pk_kind = peaks()
+    timed_s = elapsed_ms / 1e3
+    peak_key = "bf16_tflops_sustained" if timed_s >= 1.0 else "bf16_tflops"
+    peak_tf = float(pk.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    mlp1_flops = 4.0 * R * D * I
+    mlp1_tf = mlp1_flops / (mlp1_ms / 1e3) / 1e12
+    kernel_src = os.path.join(ROOT, "mixture_experts_ffn_layer_b200", "csrc", "grouped_gemm.cu")
+    traffic = traffic_from_profile(kernel_src)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights of the layer shape)",
+            "config": {"workload": "gpt-oss-20b-shaped MoE FFN layer", "T": T, "D": D, "E": E, "k": k, "I": I,
+                       "weights": "bf16", "tokens_per_gpu": T, "parallelism": f"replicas x{world} (token-sharded, "
+                       "no collective)", "l2": "inputs larger than L2 (expert weights 1.59 GB per step)"},
+            "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peak_tf, "peak_kind": f"{peak_key} ({pk_kind})",
+            "stages_ms": stage_ms,
+            "roofline": {"kernel": "grouped mlp1 (tcgen05)", "bound": "tensor", "achieved": mlp1_tf, "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": mlp1_tf / peak_tf, "traffic": traffic,
+                         "algorithmic": f"4*R*D*I = {mlp1_flops:.4g} FLOP per launch"},
+            "e2e": {"value": T * world / (e2e_ms / args.steps / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def cpu_baseline(inp, budget_s=15.0, step_tokens=None):
+    """The oracle as it stands, on the host cores, on a bounded token sample."""
+    import oracle
+
+    x = inp.x.cpu()
+    Wr, br = inp.Wr.cpu(), inp.br.cpu()
+    W1, b1, W2, b2 = inp.W1.cpu(), inp.b1.cpu(), inp.W2.cpu(), inp.b2.cpu()
+    k = inp.shape.k
+    T = x.shape[0]
+
+    def run(n, seed):
+        g = torch.Generator().manual_seed(seed)
+        toks = torch.randperm(T, generator=g)[:n]
+        xs = x[toks].contiguous()
+        t0 = time.perf_counter()
+        _, idx, w = oracle.route(xs, Wr, br, k)
+        oracle.ffn_tokens(xs, idx, w, W1, b1, W2, b2)
+        return time.perf_counter() - t0
+
+    t1 = run(2, 0)
+    n = step_tokens or max(2, min(T, int(budget_s / max(t1 / 2, 1e-6))))
+    t = run(n, 1)
+    return {"value": n / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {T} tokens of the same workload (route + top-k + softmax + expert FFN + combine per "
+                      f"token, fp64 accumulate), {t:.1f} s"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    shape = synthetic.SHAPES[WORKLOAD]
+    inp = synthetic.make_inputs(WORKLOAD, seed=synthetic.SEEDS[WORKLOAD], device="cpu")
+    x, Wr, br = inp.x, inp.Wr, inp.br
+    k, T = shape.k, shape.T
+    per_step_s = max(1.0, args.ref_budget / max(1, args.steps + args.warmup))
+
+    def one(n, seed):
+        g = torch.Generator().manual_seed(seed)
+        toks = torch.randperm(T, generator=g)[:n]
+        xs = x[toks].contiguous()
+        t0 = time.perf_counter()
+        _, idx, w = oracle.route(xs, Wr, br, k)
+        oracle.ffn_tokens(xs, idx, w, inp.W1, inp.b1, inp.W2, inp.b2)
+        return time.perf_counter() - t0
+
+    t1 = one(2, 0)
+    n = max(1, min(T, int(per_step_s / max(t1 / 2, 1e-6))))
+    for i in range(args.warmup):
+        one(n, 100 + i)
+    total = 0.0
+    for i in range(args.steps):
+        total += one(n, 1000 + i)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": "gpt-oss-20b-shaped MoE FFN layer", "T": T, "D": shape.D, "E": shape.E, "k": k,
+                   "I": shape.I, "weights": "bf16"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{n} of {T} tokens per step (route + FFN + combine per token)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

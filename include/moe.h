@@ -1,0 +1,165 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) GPT-OSS-style MoE feed-forward layer.
+ *
+ * The layer (per token t of x, T x D):
+ *   logits = x[t] . Wr^T + br                       router linear with bias
+ *   idx    = the k largest logits, ordered by (logit desc, expert index asc)
+ *   w      = softmax over those k logits
+ *   for each chosen expert e = idx[j]:
+ *     u    = W1[e] . x[t] + b1[e]                   mlp1, 2I outputs
+ *     h    = silu(u[0:I]) * u[I:2I]                 SwiGLU, rounded to bf16
+ *     o_j  = W2[e] . h + b2[e]                      mlp2, D outputs
+ *   y[t]   = sum_j w_j * o_j                        weighted combine, bf16
+ * Sources: the torchtitan GPT-OSS guide (sections "grouped matrix
+ * multiplication" -- mlp1/mlp2 as grouped GEMMs over per-expert token
+ * segments with offsets = cumsum(num_tokens_per_expert), weights stored
+ * (num_experts, out_dim, in_dim), and "HuggingFace weight adapter" -- router
+ * gate weight and bias, MXFP4 expert blocks); the from-scratch GPT-OSS
+ * write-up ("model flow" diagram: expert routing top-4, expert compute,
+ * weighted combination); the GPT-OSS in Transformers blog (MXFP4 paragraph:
+ * E2M1 values with one scale per 32-element block).
+ *
+ * Conventions for every entry point:
+ *  - All pointers are DEVICE pointers unless stated otherwise; every tensor
+ *    is dense, row-major, and at least 16-byte aligned. bf16 tensors are
+ *    passed as uint16_t bit patterns.
+ *  - The caller owns every buffer and the stream. The library allocates
+ *    nothing; scratch lives in the caller's workspace `ws` of `ws_bytes`
+ *    bytes (at least moe_workspace_bytes(d)), zero-filled once before its
+ *    first use. One workspace serves one stream at a time.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls
+ *    only enqueue work: no host synchronisation, counts stay on the device.
+ *  - Argument errors are returned synchronously (nothing is enqueued).
+ *    Errors found on the device (an index out of range, a bounded wait that
+ *    gave up) are recorded in a status word inside `ws` and read with
+ *    moe_read_device_status(); when one is recorded the outputs are
+ *    unspecified, but every memory access stayed inside the given buffers.
+ *  - Supported sizes: T >= 1, 1 <= k <= E <= 256, k <= 8, D and I multiples
+ *    of 64, D <= 16384, I <= 16384, T*k < 2^31. Other sizes return
+ *    MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, k > E, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,   /* sizes outside the supported set above */
+  MOE_ERR_WORKSPACE = 3,     /* ws_bytes < moe_workspace_bytes(d) */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  MOE_ERR_TIMEOUT = 5,       /* device: a bounded wait in a kernel gave up */
+  MOE_ERR_DEVICE_BOUNDS = 6  /* device: an expert index, row index or offset out of range */
+} moe_status_t;
+
+typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1 } moe_wfmt_t;
+
+/* T tokens, D model dim, E experts, top-k, I expert intermediate dim, and the
+ * expert-weight format (moe_wfmt_t). R = T*k routed rows. */
+typedef struct {
+  int32_t T, D, E, k, I, wfmt;
+} moe_dims_t;
+
+/* An expert weight tensor of logical shape (E, N, K), K the reduction dim.
+ * MOE_W_BF16:  data = (E, N, K) bf16, scales = NULL.
+ * MOE_W_MXFP4: data = (E, N, K/2) bytes of E2M1 codes, two per byte along K
+ *              with the even element in the low nibble; scales = (E, N, K/32)
+ *              E8M0 bytes, value 2^(s-127), one per 32 consecutive K. */
+typedef struct {
+  const void* data;
+  const uint8_t* scales;
+} moe_weight_t;
+
+/* Bytes of workspace every entry point below needs for dims d (0 if d is
+ * invalid). Holds the device status word, the permutation scratch and, for
+ * moe_forward, the routed intermediates (indices, gate weights, counts,
+ * offsets, perm, inv, gathered rows, h, expert outputs). */
+MOE_API size_t moe_workspace_bytes(moe_dims_t d);
+
+/* Validate d against the supported set (MOE_OK, INVALID_ARG or UNSUPPORTED). */
+MOE_API moe_status_t moe_check_dims(moe_dims_t d);
+
+/* Router linear + top-k + softmax over the chosen logits.
+ *   x (T,D) bf16, Wr (E,D) bf16, br (E) bf16
+ *   -> topk_idx (T,k) int32, ordered by (logit desc, expert asc);
+ *      topk_w (T,k) fp32, softmax of the chosen logits (sums to 1).
+ * Logits are accumulated in fp32 from the bf16 products. */
+MOE_API moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
+                       int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Group the R = T*k assignments a = t*k + j by expert (stable in a).
+ *   topk_idx (T,k) int32
+ *   -> counts (E) int32 tokens per expert; offsets (E+1) int32 exclusive
+ *      prefix sums (offsets[0] = 0, offsets[E] = R); perm (R) int32, row r of
+ *      the expert-sorted order holds assignment perm[r]; inv (R) int32 with
+ *      inv[perm[r]] = r (inv[a] = -1 for an out-of-range index, which also
+ *      records MOE_ERR_DEVICE_BOUNDS).
+ * Deterministic: no atomics decide any output position. */
+MOE_API moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                         int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream);
+
+/* Gather the routed rows: x_perm[r] = x[perm[r] / k], x_perm (R,D) bf16. */
+MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped mlp1 + bias + SwiGLU over the expert segments of x_perm:
+ * for r in [offsets[e], offsets[e+1]):
+ *   u = W1[e] . x_perm[r] + b1[e] (fp32 accumulate), h[r,i] = bf16(silu(u[i]) * u[I+i]).
+ *   x_perm (R,D) bf16, offsets (E+1), W1 (E,2I,D), b1 (E,2I) bf16 -> h (R,I) bf16.
+ * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile). */
+MOE_API moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
+                      const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped mlp2 + bias + gate weight over the expert segments of h:
+ *   o_perm[r] = topk_w[perm[r]] * (W2[e] . h[r] + b2[e]), stored fp32.
+ *   h (R,I) bf16, perm (R), offsets (E+1), topk_w (T*k) fp32, W2 (E,D,I),
+ *   b2 (E,D) bf16 -> o_perm (R,D) fp32. The expert outputs stay fp32 so that
+ *   the combine rounds each y element to bf16 once. */
+MOE_API moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, const int32_t* offsets,
+                      const float* topk_w, moe_weight_t W2, const uint16_t* b2, float* o_perm,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* The expert FFN of all routed rows: moe_gather, moe_mlp1, moe_mlp2 with the
+ * gathered rows and h kept in ws. o_perm (R,D) fp32 as moe_mlp2. */
+MOE_API moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* perm, const int32_t* offsets,
+                             const float* topk_w, moe_weight_t W1, const uint16_t* b1, moe_weight_t W2,
+                             const uint16_t* b2, float* o_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Weighted combine back to token order (the gate weight is already applied):
+ *   y[t] = bf16( sum_{j<k} o_perm[inv[t*k+j]] ), o_perm (R,D) fp32, summed in
+ *   fp32 in j order. A gather: each output row is written once, no atomics,
+ *   bitwise deterministic. */
+MOE_API moe_status_t moe_combine(moe_dims_t d, const float* o_perm, const int32_t* inv, uint16_t* y,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer in one call: route, permute, gather, mlp1, mlp2, combine,
+ * enqueued on `stream` with every intermediate in ws.
+ *   x (T,D) bf16, Wr (E,D), br (E), W1/b1, W2/b2 as above -> y (T,D) bf16. */
+MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
+                         moe_weight_t W1, const uint16_t* b1, moe_weight_t W2, const uint16_t* b2,
+                         uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, return the device status recorded in ws since the
+ * last read (MOE_OK if none) and clear it. */
+MOE_API moe_status_t moe_read_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_str(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

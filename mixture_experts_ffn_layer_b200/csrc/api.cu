@@ -1,0 +1,234 @@
+// The C ABI of include/moe.h: argument validation, workspace layout, and the
+// enqueueing of the kernels of route.cu, permute.cu, grouped_gemm.cu and
+// mxfp4.cu on the caller's stream. No host synchronisation except in
+// moe_read_device_status.
+#include "common.cuh"
+
+#include <stdint.h>
+
+namespace moe {
+namespace {
+
+struct WsLayout {
+  size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, w1_deq, w2_deq, total;
+};
+
+WsLayout ws_layout(const moe_dims_t& d) {
+  WsLayout L{};
+  const int64_t R = static_cast<int64_t>(d.T) * d.k;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  L.block_counts = take(static_cast<size_t>(perm_blocks(R)) * d.E * 4);
+  L.topk_idx = take(R * 4);
+  L.topk_w = take(R * 4);
+  L.counts = take(static_cast<size_t>(d.E) * 4);
+  L.offsets = take(static_cast<size_t>(d.E + 1) * 4);
+  L.perm = take(R * 4);
+  L.inv = take(R * 4);
+  L.x_perm = take(static_cast<size_t>(R) * d.D * 2);
+  L.h = take(static_cast<size_t>(R) * d.I * 2);
+  L.o_perm = take(static_cast<size_t>(R) * d.D * 4);
+  if (d.wfmt == MOE_W_MXFP4) {
+    L.w1_deq = take(static_cast<size_t>(d.E) * 2 * d.I * d.D * 2);
+    L.w2_deq = take(static_cast<size_t>(d.E) * d.D * d.I * 2);
+  }
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int* status_word(void* ws) { return static_cast<int*>(ws); }
+
+moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(d).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status_t check_weight(const moe_dims_t& d, const moe_weight_t& w) {
+  if (!w.data || !aligned16(w.data)) return MOE_ERR_INVALID_ARG;
+  if (d.wfmt == MOE_W_MXFP4 && (!w.scales)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                      \
+  do {                                     \
+    moe_status_t _st = (expr);             \
+    if (_st != MOE_OK) return _st;         \
+  } while (0)
+
+#define MOE_REQUIRE(cond)                         \
+  do {                                            \
+    if (!(cond)) return MOE_ERR_INVALID_ARG;      \
+  } while (0)
+
+// bf16 view of an expert weight: the tensor itself, or its expansion in ws.
+moe_status_t weight_bf16(const moe_dims_t& d, const moe_weight_t& w, int64_t N, int64_t K, void* ws, size_t deq_off,
+                         cudaStream_t s, const uint16_t** out) {
+  if (d.wfmt == MOE_W_BF16) {
+    *out = static_cast<const uint16_t*>(w.data);
+    return MOE_OK;
+  }
+  uint16_t* deq = at<uint16_t>(ws, deq_off);
+  MOE_TRY(cuda_status(launch_dequant_mxfp4(static_cast<const uint8_t*>(w.data), w.scales, d.E, N, K, deq, s)));
+  *out = deq;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status_t moe_check_dims(moe_dims_t d) {
+  if (d.T <= 0 || d.D <= 0 || d.E <= 0 || d.k <= 0 || d.I <= 0) return MOE_ERR_INVALID_ARG;
+  if (d.k > d.E) return MOE_ERR_INVALID_ARG;
+  if (d.wfmt != MOE_W_BF16 && d.wfmt != MOE_W_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (d.E > 256 || d.k > 8) return MOE_ERR_UNSUPPORTED;
+  if (d.D % 64 || d.I % 64 || d.D > 16384 || d.I > 16384) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d.T) * d.k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(moe_dims_t d) {
+  if (moe_check_dims(d) != MOE_OK) return 0;
+  return ws_layout(d).total;
+}
+
+moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br, int32_t* topk_idx,
+                       float* topk_w, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(x && Wr && br && topk_idx && topk_w);
+  MOE_REQUIRE(aligned16(x) && aligned16(Wr));
+  return cuda_status(launch_route(d, x, Wr, br, topk_idx, topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(topk_idx && counts && offsets && perm && inv);
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  const WsLayout L = ws_layout(d);
+  return cuda_status(launch_permute(d, topk_idx, counts, offsets, perm, inv, at<int32_t>(ws, L.block_counts),
+                                    status_word(ws), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm, void* ws,
+                        size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(x && perm && x_perm && aligned16(x) && aligned16(x_perm));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  return cuda_status(launch_gather(d, x, perm, x_perm, status_word(ws), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
+                      const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(x_perm && offsets && b1 && h && aligned16(x_perm) && aligned16(b1) && aligned16(h));
+  MOE_TRY(check_weight(d, W1));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(d);
+  const uint16_t* w1 = nullptr;
+  MOE_TRY(weight_bf16(d, W1, 2 * static_cast<int64_t>(d.I), d.D, ws, L.w1_deq, s, &w1));
+  return launch_mlp1(d, x_perm, offsets, w1, b1, h, status_word(ws), s);
+}
+
+moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, const int32_t* offsets,
+                      const float* topk_w, moe_weight_t W2, const uint16_t* b2, float* o_perm, void* ws,
+                      size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(h && perm && offsets && topk_w && b2 && o_perm && aligned16(h) && aligned16(b2) && aligned16(o_perm));
+  MOE_TRY(check_weight(d, W2));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(d);
+  const uint16_t* w2 = nullptr;
+  MOE_TRY(weight_bf16(d, W2, d.D, d.I, ws, L.w2_deq, s, &w2));
+  return launch_mlp2(d, h, perm, offsets, topk_w, w2, b2, o_perm, status_word(ws), s);
+}
+
+moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* perm, const int32_t* offsets,
+                             const float* topk_w, moe_weight_t W1, const uint16_t* b1, moe_weight_t W2,
+                             const uint16_t* b2, float* o_perm, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(x && perm && offsets && topk_w && b1 && b2 && o_perm);
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  const WsLayout L = ws_layout(d);
+  uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  MOE_TRY(moe_gather(d, x, perm, x_perm, ws, ws_bytes, stream));
+  MOE_TRY(moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, ws_bytes, stream));
+  return moe_mlp2(d, h, perm, offsets, topk_w, W2, b2, o_perm, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_combine(moe_dims_t d, const float* o_perm, const int32_t* inv, uint16_t* y, void* ws,
+                         size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(o_perm && inv && y && aligned16(o_perm) && aligned16(y));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  return cuda_status(launch_combine(d, o_perm, inv, y, status_word(ws), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br, moe_weight_t W1,
+                         const uint16_t* b1, moe_weight_t W2, const uint16_t* b2, uint16_t* y, void* ws,
+                         size_t ws_bytes, void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(x && Wr && br && b1 && b2 && y);
+  MOE_TRY(check_weight(d, W1));
+  MOE_TRY(check_weight(d, W2));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  const WsLayout L = ws_layout(d);
+  int32_t* topk_idx = at<int32_t>(ws, L.topk_idx);
+  float* topk_w = at<float>(ws, L.topk_w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  float* o_perm = at<float>(ws, L.o_perm);
+  MOE_TRY(moe_route(d, x, Wr, br, topk_idx, topk_w, stream));
+  MOE_TRY(moe_permute(d, topk_idx, counts, offsets, perm, inv, ws, ws_bytes, stream));
+  MOE_TRY(moe_ffn_grouped(d, x, perm, offsets, topk_w, W1, b1, W2, b2, o_perm, ws, ws_bytes, stream));
+  return moe_combine(d, o_perm, inv, y, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_read_device_status(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0) {
+    if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return static_cast<moe_status_t>(v);
+}
+
+const char* moe_status_str(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported sizes";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_TIMEOUT: return "device: bounded wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "device: index or offset out of range";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

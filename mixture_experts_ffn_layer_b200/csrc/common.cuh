@@ -1,0 +1,67 @@
+// Shared device/host helpers of the MoE layer's CUDA path.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Workspace header: the device status word lives at byte 0 of ws.
+constexpr size_t kWsHeader = 256;
+
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(float_to_bf16_bits(lo)) | (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
+}
+
+// Launch helpers shared by the host side of every .cu file.
+struct Launch {
+  cudaStream_t stream;
+  int* status;  // device status word (may be null for kernels that never record)
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Permutation block size: assignments per histogram/scatter block.
+constexpr int kPermChunk = 2048;
+constexpr int kPermThreads = 256;
+
+inline int perm_blocks(int64_t R) { return static_cast<int>((R + kPermChunk - 1) / kPermChunk); }
+
+// Kernel launchers (defined in the .cu files).
+cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t s);
+cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                           int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s);
+cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
+                          int* status, cudaStream_t s);
+cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32_t* inv, uint16_t* y,
+                           int* status, cudaStream_t s);
+
+// Grouped GEMMs (grouped_gemm.cu). Return MOE_OK or an error code.
+moe_status_t launch_mlp1(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
+                         const uint16_t* W1, const uint16_t* b1, uint16_t* h, int* status, cudaStream_t s);
+moe_status_t launch_mlp2(const moe_dims_t& d, const uint16_t* h, const int32_t* perm, const int32_t* offsets,
+                         const float* topk_w, const uint16_t* W2, const uint16_t* b2, float* o_perm,
+                         int* status, cudaStream_t s);
+
+// MXFP4 -> bf16 expansion of an (E, N, K) expert weight (mxfp4.cu).
+cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t E, int64_t N, int64_t K,
+                                 uint16_t* out, cudaStream_t s);
+
+}  // namespace moe

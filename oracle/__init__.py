@@ -50,7 +50,7 @@ def lib():
         L.oracle_route.argtypes = [c_i64, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
         L.oracle_permute.argtypes = [c_i64, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]
         L.oracle_ffn_tokens.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp,
-                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp]
+                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp]
         L.oracle_forward.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
         for f in ("oracle_dequant_mxfp4", "oracle_route", "oracle_permute", "oracle_ffn_tokens", "oracle_forward"):
@@ -121,9 +121,10 @@ def permute(topk_idx, E: int):
 
 
 def ffn_tokens(x, topk_idx, topk_w, W1, b1, W2, b2, tokens: Optional[Sequence[int]] = None,
-               W1_scales=None, W2_scales=None, return_o: bool = False):
+               W1_scales=None, W2_scales=None, return_o: bool = False, return_exact: bool = False):
     """Expert FFN + weighted combine for ``tokens`` (default all) -> y (n, D) bf16
-    [and o (n, k, D) float64, the unweighted expert outputs]."""
+    [and o (n, k, D) float64, the unweighted expert outputs]
+    [and y_exact (n, D) float64, y before its final bf16 rounding]."""
     x, idx, w = _cpu(x), _cpu(topk_idx).to(torch.int32), _cpu(topk_w).float()
     W1, b1, W2, b2 = _cpu(W1), _cpu(b1), _cpu(W2), _cpu(b2)
     W1s, W2s = _cpu(W1_scales), _cpu(W2_scales)
@@ -139,10 +140,16 @@ def ffn_tokens(x, topk_idx, topk_w, W1, b1, W2, b2, tokens: Optional[Sequence[in
     n = tok.numel()
     y = torch.empty((n, D), dtype=torch.int16)
     o = torch.empty((n, k, D), dtype=torch.float64) if return_o else None
+    ye = torch.empty((n, D), dtype=torch.float64) if return_exact else None
     _check(lib().oracle_ffn_tokens(T, D, E, k, I, wfmt, _ptr(x), _ptr(idx), _ptr(w), _ptr(W1), _ptr(W1s), _ptr(b1),
-                                   _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(tok), n, _ptr(y), _ptr(o)), "ffn_tokens")
-    y = y.view(torch.bfloat16)
-    return (y, o) if return_o else y
+                                   _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(tok), n, _ptr(y), _ptr(o), _ptr(ye)),
+           "ffn_tokens")
+    out = [y.view(torch.bfloat16)]
+    if return_o:
+        out.append(o)
+    if return_exact:
+        out.append(ye)
+    return tuple(out) if len(out) > 1 else out[0]
 
 
 def forward(x, Wr, br, W1, b1, W2, b2, k: int, W1_scales=None, W2_scales=None):

@@ -219,11 +219,12 @@ int oracle_permute(int64_t T, int E, int k, const int32_t* topk_idx, int32_t* co
 // wfmt 0: W1 (E,2I,D) and W2 (E,D,I) are bf16. wfmt 1: they are MXFP4 codes
 // (E,2I,D/2), (E,D,I/2) with scales (E,2I,D/32), (E,D,I/32).
 // y_out: ntok x D bf16. o_out (nullable): ntok x k x D doubles, the unweighted
-// expert outputs o_j.
+// expert outputs o_j. y_exact (nullable): ntok x D doubles, the weighted sum
+// before its final bf16 rounding.
 int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, const uint16_t* x,
                       const int32_t* topk_idx, const float* topk_w, const void* W1, const uint8_t* W1_scales,
                       const uint16_t* b1, const void* W2, const uint8_t* W2_scales, const uint16_t* b2,
-                      const int64_t* tokens, int64_t ntok, uint16_t* y_out, double* o_out) {
+                      const int64_t* tokens, int64_t ntok, uint16_t* y_out, double* o_out, double* y_exact) {
   if (!dims_ok(T, D, E, k, I)) return 1;
   if (wfmt != 0 && wfmt != 1) return 1;
   if (wfmt == 1 && (D % 32 || I % 32)) return 1;
@@ -256,6 +257,8 @@ int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, const uin
           for (int c = 0; c < D; ++c) o_out[(s * k + j) * D + c] = o[c];
       }
       for (int c = 0; c < D; ++c) y_out[s * D + c] = double_to_bf16(y[c]);
+      if (y_exact)
+        for (int c = 0; c < D; ++c) y_exact[s * D + c] = y[c];
     }
   }
   return err;
@@ -271,7 +274,7 @@ int oracle_forward(int64_t T, int D, int E, int k, int I, int wfmt, const uint16
   std::vector<int64_t> tokens(T);
   for (int64_t t = 0; t < T; ++t) tokens[t] = t;
   return oracle_ffn_tokens(T, D, E, k, I, wfmt, x, topk_idx, topk_w, W1, W1_scales, b1, W2, W2_scales, b2,
-                           tokens.data(), T, y, nullptr);
+                           tokens.data(), T, y, nullptr, nullptr);
 }
 
 }  // extern "C"

@@ -1,0 +1,74 @@
+"""The C-ABI library: it builds, loads, exports every symbol include/moe.h
+declares, and its host-side logic (size validation, workspace sizing,
+synchronous argument errors) works without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_ffn_layer_b200 as moe
+from mixture_experts_ffn_layer_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.load()
+    names = _declared()
+    assert len(names) >= 12
+    assert sorted(_binding.EXPORTS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+    # nothing but the C ABI is exported
+    out = os.popen(f"nm -D --defined-only {_binding.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r" T (moe_\w+)", out)))
+    assert exported == names
+
+
+def test_check_dims_supported_set():
+    ok = moe.dims(8192, 2880, 32, 4, 2880)
+    assert moe.check_dims(ok) == 0
+    assert moe.check_dims(moe.dims(0, 64, 4, 2, 64)) == 1  # T = 0
+    assert moe.check_dims(moe.dims(8, 64, 4, 5, 64)) == 1  # k > E
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, wfmt=7)) == 1
+    assert moe.check_dims(moe.dims(8, 64, 300, 2, 64)) == 2  # E > 256
+    assert moe.check_dims(moe.dims(8, 64, 16, 9, 64)) == 2  # k > 8
+    assert moe.check_dims(moe.dims(8, 96, 4, 2, 64)) == 2  # D % 64
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 100)) == 2  # I % 64
+
+
+def test_workspace_bytes_covers_intermediates():
+    d = moe.dims(8192, 2880, 32, 4, 2880)
+    R = 8192 * 4
+    n = moe.workspace_bytes(d)
+    need = R * 2880 * (2 + 2 + 4) + R * 4 * 4  # x_perm, h (bf16), o_perm (fp32) + idx, w, perm, inv
+    assert need <= n <= need + 4 * 1024 * 1024
+    dq = moe.dims(8192, 2880, 32, 4, 2880, wfmt=moe.MOE_W_MXFP4)
+    assert moe.workspace_bytes(dq) - n >= 32 * 3 * 2880 * 2880 * 2  # dequantized W1 and W2
+    with pytest.raises(moe.MoeError):
+        moe.workspace_bytes(moe.dims(8, 64, 4, 5, 64))
+
+
+def test_argument_errors_are_synchronous():
+    lib = moe.load()
+    d = moe.dims(64, 64, 4, 2, 64)
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: validation fails first
+    assert lib.moe_route(d, None, fake, fake, fake, fake, None) == 1
+    assert lib.moe_route(d, vp((1 << 20) + 8), fake, fake, fake, fake, None) == 1  # misaligned x
+    assert lib.moe_permute(d, fake, fake, fake, fake, fake, fake, 16, None) == 3  # workspace too small
+    assert lib.moe_permute(d, fake, fake, fake, fake, fake, vp((1 << 20) + 4), 1 << 30, None) == 1
+    w = _binding.Weight(None, None)
+    assert lib.moe_mlp1(d, fake, fake, w, fake, fake, fake, 1 << 30, None) == 1
+    dq = moe.dims(64, 64, 4, 2, 64, wfmt=moe.MOE_W_MXFP4)
+    wq = _binding.Weight(1 << 20, None)  # MXFP4 without scales
+    assert lib.moe_mlp1(dq, fake, fake, wq, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.moe_forward(moe.dims(64, 64, 4, 9, 64), fake, fake, fake, w, fake, w, fake, fake, fake, 0, None) == 1
+    assert lib.moe_read_device_status(None, None) == 1
+    assert moe.status_str(6) == "device: index or offset out of range"

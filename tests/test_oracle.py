@@ -220,6 +220,17 @@ def test_ffn_matches_dense_all_expert_brute_force(T, D, E, k, I):
     np.testing.assert_allclose(y.double().numpy(), y_dense, rtol=2 ** -7, atol=1e-5)
 
 
+def test_exact_output_rounds_to_output():
+    T, D, E, k, I = 16, 64, 4, 2, 32
+    inp = synthetic.make_custom(T, D, E, k, I, seed=12)
+    _, idx, w = oracle.route(inp.x, inp.Wr, inp.br, k)
+    y, o, ye = oracle.ffn_tokens(inp.x, idx, w, inp.W1, inp.b1, inp.W2, inp.b2, return_o=True, return_exact=True)
+    assert torch.equal(oracle.round_bf16(ye).view(torch.int16), y.view(torch.int16))
+    # y_exact is the gate-weighted sum of the expert outputs
+    ref = (w.double()[:, :, None] * o).sum(1)
+    assert torch.allclose(ye, ref, rtol=1e-14, atol=1e-15)
+
+
 def test_w2_zero_gives_weighted_bias_sum():
     T, D, E, k, I = 16, 32, 6, 3, 16
     inp = synthetic.make_custom(T, D, E, k, I, seed=2)
