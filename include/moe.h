@@ -95,9 +95,10 @@ MOE_API moe_status_t moe_check_dims(moe_dims_t d);
  *   x (T,D) bf16, Wr (E,D) bf16, br (E) bf16
  *   -> topk_idx (T,k) int32, ordered by (logit desc, expert asc);
  *      topk_w (T,k) fp32, softmax of the chosen logits (sums to 1).
- * Logits are accumulated in fp32 from the bf16 products. */
+ * Logits are accumulated in fp32 from the bf16 products (tcgen05 tensor
+ * cores, one 128-token tile per CTA); ws holds only the status word. */
 MOE_API moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
-                       int32_t* topk_idx, float* topk_w, void* stream);
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
 /* Group the R = T*k assignments a = t*k + j by expert (stable in a).
  *   topk_idx (T,k) int32

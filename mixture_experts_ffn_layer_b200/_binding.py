@@ -59,7 +59,7 @@ def load(path: str = LIB_PATH):
     sig = {
         "moe_workspace_bytes": (ctypes.c_size_t, [Dims]),
         "moe_check_dims": (ctypes.c_int, [Dims]),
-        "moe_route": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP]),
+        "moe_route": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_permute": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_gather": (ctypes.c_int, [Dims, VP, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_mlp1": (ctypes.c_int, [Dims, VP, VP, Weight, VP, VP, VP, ctypes.c_size_t, VP]),
@@ -116,8 +116,9 @@ def check_dims(d: Dims) -> int:
     return load().moe_check_dims(d)
 
 
-def moe_route(d, x, Wr, br, topk_idx, topk_w, stream=None):
-    _check(load().moe_route(d, _p(x), _p(Wr), _p(br), _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route")
+def moe_route(d, x, Wr, br, topk_idx, topk_w, ws, stream=None):
+    _check(load().moe_route(d, _p(x), _p(Wr), _p(br), _p(topk_idx), _p(topk_w), _p(ws), ws.numel(), _stream(stream)),
+           "moe_route")
 
 
 def moe_permute(d, topk_idx, counts, offsets, perm, inv, ws, stream=None):

@@ -110,11 +110,13 @@ size_t moe_workspace_bytes(moe_dims_t d) {
 }
 
 moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br, int32_t* topk_idx,
-                       float* topk_w, void* stream) {
+                       float* topk_w, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
   MOE_REQUIRE(x && Wr && br && topk_idx && topk_w);
   MOE_REQUIRE(aligned16(x) && aligned16(Wr));
-  return cuda_status(launch_route(d, x, Wr, br, topk_idx, topk_w, static_cast<cudaStream_t>(stream)));
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  return cuda_status(
+      launch_route(d, x, Wr, br, topk_idx, topk_w, status_word(ws), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets, int32_t* perm,
@@ -200,7 +202,7 @@ moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, co
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* inv = at<int32_t>(ws, L.inv);
   float* o_perm = at<float>(ws, L.o_perm);
-  MOE_TRY(moe_route(d, x, Wr, br, topk_idx, topk_w, stream));
+  MOE_TRY(moe_route(d, x, Wr, br, topk_idx, topk_w, ws, ws_bytes, stream));
   MOE_TRY(moe_permute(d, topk_idx, counts, offsets, perm, inv, ws, ws_bytes, stream));
   MOE_TRY(moe_ffn_grouped(d, x, perm, offsets, topk_w, W1, b1, W2, b2, o_perm, ws, ws_bytes, stream));
   return moe_combine(d, o_perm, inv, y, ws, ws_bytes, stream);

@@ -45,7 +45,7 @@ inline int perm_blocks(int64_t R) { return static_cast<int>((R + kPermChunk - 1)
 
 // Kernel launchers (defined in the .cu files).
 cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
-                         int32_t* topk_idx, float* topk_w, cudaStream_t s);
+                         int32_t* topk_idx, float* topk_w, int* status, cudaStream_t s);
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s);
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,

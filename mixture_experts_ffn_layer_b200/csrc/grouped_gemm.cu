@@ -28,8 +28,7 @@
 // frees TMEM and returns.
 #include "common.cuh"
 #include "sm100.cuh"
-
-#include <cudaTypedefs.h>
+#include "tma_host.cuh"
 
 namespace moe {
 namespace {
@@ -294,32 +293,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = static_cast<int64_t>(seg[e]) + mt * BM + row_in_tile;
       const bool valid = row < seg[e + 1];
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccStride;
+      // Columns are drained 32 at a time: up to four 8-column TMEM loads per
+      // wait (the bounds are warp-uniform, as tcgen05.ld requires).
       if (kSwiGLU) {
         const uint16_t* bg = p.bias + static_cast<int64_t>(e) * p.b_rows + nt * p.n_tile;
         const uint16_t* bu = bg + p.n_out;
         uint16_t* dst = static_cast<uint16_t*>(p.out) + row * p.n_out + nt * p.n_tile;
-        for (int c = 0; c < p.n_tile; c += 8) {
-          uint32_t g[8], u[8];
-          tmem_ld_x8(tbase + c, g);
-          tmem_ld_x8(tbase + p.n_tile + c, u);
-          tmem_ld_wait();
-          float gb[8], ub[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(bg + c)), gb);
-          unpack8(__ldg(reinterpret_cast<const uint4*>(bu + c)), ub);
-          float hv[8];
+        for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+          uint32_t g[32], u[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float gate = __uint_as_float(g[i]) + gb[i];
-            const float up = __uint_as_float(u[i]) + ub[i];
-            hv[i] = __fdividef(gate, 1.0f + __expf(-gate)) * up;
+          for (int j = 0; j < 4; ++j) {
+            if (c0 + 8 * j < p.n_tile) {
+              tmem_ld_x8(tbase + c0 + 8 * j, g + 8 * j);
+              tmem_ld_x8(tbase + p.n_tile + c0 + 8 * j, u + 8 * j);
+            }
           }
-          if (valid) {
-            uint4 v;
-            v.x = pack_bf16x2(hv[0], hv[1]);
-            v.y = pack_bf16x2(hv[2], hv[3]);
-            v.z = pack_bf16x2(hv[4], hv[5]);
-            v.w = pack_bf16x2(hv[6], hv[7]);
-            *reinterpret_cast<uint4*>(dst + c) = v;
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = c0 + 8 * j;
+            if (c < p.n_tile) {
+              float gb[8], ub[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(bg + c)), gb);
+              unpack8(__ldg(reinterpret_cast<const uint4*>(bu + c)), ub);
+              float hv[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float gate = __uint_as_float(g[8 * j + i]) + gb[i];
+                const float up = __uint_as_float(u[8 * j + i]) + ub[i];
+                hv[i] = __fdividef(gate, 1.0f + __expf(-gate)) * up;
+              }
+              if (valid) {
+                uint4 v;
+                v.x = pack_bf16x2(hv[0], hv[1]);
+                v.y = pack_bf16x2(hv[2], hv[3]);
+                v.z = pack_bf16x2(hv[4], hv[5]);
+                v.w = pack_bf16x2(hv[6], hv[7]);
+                *reinterpret_cast<uint4*>(dst + c) = v;
+              }
+            }
           }
         }
       } else {
@@ -333,24 +345,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint16_t* bb = p.bias + static_cast<int64_t>(e) * p.b_rows + nt * p.n_tile;
         float* dst = static_cast<float*>(p.out) + row * p.n_out + nt * p.n_tile;
-        for (int c = 0; c < p.n_tile; c += 8) {
-          uint32_t v8[8];
-          tmem_ld_x8(tbase + c, v8);
+        for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+          uint32_t v[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (c0 + 8 * j < p.n_tile) tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
           tmem_ld_wait();
-          float bv[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(bb + c)), bv);
-          float4 o0, o1;
-          o0.x = wgt * (__uint_as_float(v8[0]) + bv[0]);
-          o0.y = wgt * (__uint_as_float(v8[1]) + bv[1]);
-          o0.z = wgt * (__uint_as_float(v8[2]) + bv[2]);
-          o0.w = wgt * (__uint_as_float(v8[3]) + bv[3]);
-          o1.x = wgt * (__uint_as_float(v8[4]) + bv[4]);
-          o1.y = wgt * (__uint_as_float(v8[5]) + bv[5]);
-          o1.z = wgt * (__uint_as_float(v8[6]) + bv[6]);
-          o1.w = wgt * (__uint_as_float(v8[7]) + bv[7]);
-          if (valid) {
-            reinterpret_cast<float4*>(dst + c)[0] = o0;
-            reinterpret_cast<float4*>(dst + c)[1] = o1;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = c0 + 8 * j;
+            if (c < p.n_tile) {
+              float bv[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(bb + c)), bv);
+              float4 o0, o1;
+              o0.x = wgt * (__uint_as_float(v[8 * j + 0]) + bv[0]);
+              o0.y = wgt * (__uint_as_float(v[8 * j + 1]) + bv[1]);
+              o0.z = wgt * (__uint_as_float(v[8 * j + 2]) + bv[2]);
+              o0.w = wgt * (__uint_as_float(v[8 * j + 3]) + bv[3]);
+              o1.x = wgt * (__uint_as_float(v[8 * j + 4]) + bv[4]);
+              o1.y = wgt * (__uint_as_float(v[8 * j + 5]) + bv[5]);
+              o1.z = wgt * (__uint_as_float(v[8 * j + 6]) + bv[6]);
+              o1.w = wgt * (__uint_as_float(v[8 * j + 7]) + bv[7]);
+              if (valid) {
+                reinterpret_cast<float4*>(dst + c)[0] = o0;
+                reinterpret_cast<float4*>(dst + c)[1] = o1;
+              }
+            }
           }
         }
       }
@@ -373,43 +393,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2-D bf16 tensor (rows x inner), K-major tiles of 64 x box_rows, 128-byte swizzle.
-bool make_tmap(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-int num_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
-
 int pick_tile(int n, int max_tile, int step) {
   for (int t = max_tile; t >= step; t -= step)
     if (n % t == 0) return t;
@@ -440,8 +423,8 @@ moe_status_t launch_mlp1(const moe_dims_t& d, const uint16_t* x_perm, const int3
   const int nh = pick_tile(d.I, 128, 8);
   if (nh == 0) return MOE_ERR_UNSUPPORTED;
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, x_perm, d.D, R, BM)) return MOE_ERR_CUDA;
-  if (!make_tmap(&tb, W1, d.D, static_cast<uint64_t>(d.E) * 2 * d.I, nh)) return MOE_ERR_CUDA;
+  if (!make_tmap_bf16(&ta, x_perm, d.D, R, BM)) return MOE_ERR_CUDA;
+  if (!make_tmap_bf16(&tb, W1, d.D, static_cast<uint64_t>(d.E) * 2 * d.I, nh)) return MOE_ERR_CUDA;
   GemmParams p{};
   p.E = d.E;
   p.K = d.D;
@@ -465,8 +448,8 @@ moe_status_t launch_mlp2(const moe_dims_t& d, const uint16_t* h, const int32_t* 
   const int nt = pick_tile(d.D, 256, 16);
   if (nt == 0) return MOE_ERR_UNSUPPORTED;
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, h, d.I, R, BM)) return MOE_ERR_CUDA;
-  if (!make_tmap(&tb, W2, d.I, static_cast<uint64_t>(d.E) * d.D, nt)) return MOE_ERR_CUDA;
+  if (!make_tmap_bf16(&ta, h, d.I, R, BM)) return MOE_ERR_CUDA;
+  if (!make_tmap_bf16(&tb, W2, d.I, static_cast<uint64_t>(d.E) * d.D, nt)) return MOE_ERR_CUDA;
   GemmParams p{};
   p.E = d.E;
   p.K = d.I;

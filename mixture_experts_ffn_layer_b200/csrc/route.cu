@@ -1,160 +1,254 @@
-// Router linear + top-k + softmax over the chosen logits.
+// Router linear + top-k + softmax over the chosen logits, on the tensor cores.
 //
 // The router is a linear layer with bias (torchtitan GPT-OSS guide, HuggingFace
 // weight adapter section: moe.router.gate.weight/bias); the from-scratch GPT-OSS
 // write-up's model flow routes each token to its top-4 experts. Gate weights
 // are the softmax of the k chosen logits; ties go to the lower expert index.
 //
-// One CTA handles kTok tokens: the logits tile (kTok x E) is accumulated in
-// fp32 registers from bf16 tiles of x and Wr staged in shared memory, then one
-// warp per token selects the top k with warp shuffles and writes the
-// normalised weights. HBM traffic is x once plus Wr (L2-resident).
+// The logits are a dense contraction (T x D) . (D x E), so each CTA computes a
+// 128-token tile of them with tcgen05.mma (M=128, N=E rounded up to 16, K=D)
+// into TMEM, fed by TMA (x rows and all of Wr, 64-wide K slices, 128-byte
+// swizzle, 4-stage ring). Its epilogue is one thread per token (= TMEM lane):
+// it streams the token's E logits out of TMEM, adds the bias, keeps a sorted
+// top-k in registers and writes the normalised gate weights. x is read once
+// from HBM; Wr stays L2-resident.
 #include "common.cuh"
+#include "sm100.cuh"
+#include "tma_host.cuh"
 
 #include <float.h>
 
 namespace moe {
 namespace {
 
-constexpr int kTok = 32;      // tokens per CTA
-constexpr int kDc = 32;       // reduction chunk staged in shared memory
-constexpr int kThreads = 256; // 16 x 16 thread grid: tokens x expert groups
+using namespace sm100;
 
-template <int EJ>  // experts per thread: E <= 16 * EJ
-__global__ void __launch_bounds__(kThreads) route_kernel(int T, int D, int E, int k, const uint16_t* __restrict__ x,
-                                                         const uint16_t* __restrict__ Wr,
-                                                         const uint16_t* __restrict__ br, int32_t* __restrict__ topk_idx,
-                                                         float* __restrict__ topk_w) {
-  constexpr int EP = 16 * EJ;
-  constexpr int kWsFloats = EP * (kDc + 1), kLgFloats = kTok * (EP + 1);
-  __shared__ float xs[kTok][kDc + 1];
-  // The Wr tile and, after the reduction, the logits tile share this buffer.
-  __shared__ float buf[kWsFloats > kLgFloats ? kWsFloats : kLgFloats];
-  float (*ws)[kDc + 1] = reinterpret_cast<float (*)[kDc + 1]>(buf);
-  float (*lg)[EP + 1] = reinterpret_cast<float (*)[EP + 1]>(buf);
+constexpr int BM = 128, BK = 64, kStages = 4, kThreads = 192, kMaxK = 8;
+constexpr int kABytes = BM * BK * 2;
+constexpr uint64_t kWaitNs = 1000000000ull;
 
-  const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;
-  const int t0 = blockIdx.x * kTok;
+struct RouteParams {
+  int T, D, E, k;
+  int n_pad;        // MMA N: E rounded up to a multiple of 16
+  uint32_t tmem_cols;
+  const uint16_t* br;
+  int32_t* topk_idx;
+  float* topk_w;
+  int* status;
+};
 
-  float acc[2][EJ];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) acc[i][j] = 0.f;
+__global__ void __launch_bounds__(kThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const RouteParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t stage_bytes = kABytes + p.n_pad * BK * 2;
+  uint8_t* ctrl = smem + kStages * stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);  // full[S] empty[S] tfull done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * kStages + 2));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  for (int d0 = 0; d0 < D; d0 += kDc) {
-    // x tile: kTok x kDc bf16 = 128 vectors of 8
-    if (tid < kTok * kDc / 8) {
-      int r = tid / (kDc / 8), c = (tid % (kDc / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + r < T) v = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t0 + r) * D + d0 + c);
-      const uint16_t* p = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) xs[r][c + q] = bf16_bits_to_float(p[q]);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * kStages);
+  const uint32_t done_bar = bar0 + 8u * (2 * kStages + 1);
+  const int t0 = blockIdx.x * BM;
+  const int KB = (p.D + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
     }
-    // Wr tile: EP x kDc
-    for (int v_id = tid; v_id < EP * kDc / 8; v_id += kThreads) {
-      int r = v_id / (kDc / 8), c = (v_id % (kDc / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < E) v = *reinterpret_cast<const uint4*>(Wr + static_cast<int64_t>(r) * D + d0 + c);
-      const uint16_t* p = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) ws[r][c + q] = bf16_bits_to_float(p[q]);
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int dd = 0; dd < kDc; ++dd) {
-      float xv0 = xs[ty][dd], xv1 = xs[ty + 16][dd];
-#pragma unroll
-      for (int j = 0; j < EJ; ++j) {
-        float wv = ws[tx + 16 * j][dd];
-        acc[0][j] = fmaf(xv0, wv, acc[0][j]);
-        acc[1][j] = fmaf(xv1, wv, acc[1][j]);
-      }
-    }
-    __syncthreads();
+    mbar_init(tfull_bar, 1);
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
   }
-#pragma unroll
-  for (int j = 0; j < EJ; ++j) {
-    int e = tx + 16 * j;
-    float b = e < E ? bf16_bits_to_float(br[e]) : 0.f;
-    lg[ty][e] = acc[0][j] + b;
-    lg[ty + 16][e] = acc[1][j] + b;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+    tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  // Top-k: one warp per token, lanes own experts lane, lane+32, ...
-  const int warp = tid / 32, lane = tid % 32;
-  constexpr int kPer = (EP + 31) / 32;
-  for (int r = warp; r < kTok; r += kThreads / 32) {
-    const int t = t0 + r;
-    if (t >= T) break;
-    float v[kPer];
-#pragma unroll
-    for (int m = 0; m < kPer; ++m) {
-      int e = lane + 32 * m;
-      v[m] = e < E ? lg[r][e] : -FLT_MAX;
-    }
-    bool taken[kPer];
-#pragma unroll
-    for (int m = 0; m < kPer; ++m) taken[m] = (lane + 32 * m) >= E;
-    float sel_v = 0.f, v0 = 0.f, denom = 0.f;
-    int sel_e = 0;
-    for (int j = 0; j < k; ++j) {
-      // local best among untaken: (value desc, index asc)
-      float bv = -FLT_MAX;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        int e = lane + 32 * m;
-        if (!taken[m] && (v[m] > bv || (v[m] == bv && e < be))) {
-          bv = v[m];
-          be = e;
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool failed = false;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, kWaitNs)) {
+          failed = true;
+          break;
+        }
+        const uint32_t a_dst = smem_u32(smem + stage * stage_bytes);
+        mbar_arrive_expect_tx(full_bar(stage), stage_bytes);
+        tma_load_2d(a_dst, &tmX, full_bar(stage), kb * BK, t0);
+        tma_load_2d(a_dst + kABytes, &tmW, full_bar(stage), kb * BK, 0);
+        ++issued;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
+      if (failed) {
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        const int n = issued < kStages ? issued : kStages;
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = kStages - 1;
+            ph ^= 1u;
+          }
+          mbar_wait_bounded(full_bar(s), ph, nullptr, kWaitNs);
         }
       }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer: one 128 x n_pad accumulator over all of K
+      const uint32_t idesc = idesc_bf16_f32(BM, p.n_pad);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool failed = false;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, kWaitNs)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * stage_bytes);
+        const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
-      for (int m = 0; m < kPer; ++m)
-        if (lane + 32 * m == be) taken[m] = true;
-      if (j == 0) v0 = bv;
-      float ex = __expf(bv - v0);
-      denom += ex;
-      if (lane == j) {
-        sel_v = ex;
-        sel_e = be;
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16(tmem_base, desc_kmajor_sw128(a_addr + kk * 32), desc_kmajor_sw128(b_addr + kk * 32), idesc,
+                   (kb | kk) != 0 ? 1u : 0u);
+        tc_commit(empty_bar(stage));
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
+      if (failed) {
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+      } else {
+        tc_commit(tfull_bar);
+      }
+      tc_commit(done_bar);
+      mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
     }
-    if (lane < k) {
-      topk_idx[static_cast<int64_t>(t) * k + lane] = sel_e;
-      topk_w[static_cast<int64_t>(t) * k + lane] = sel_v / denom;
+  } else {
+    // epilogue: thread = token = TMEM lane
+    const int q = warp & 3;
+    const int t = t0 + q * 32 + lane;
+    const bool ok = mbar_wait_bounded(tfull_bar, 0, abort_flag, kWaitNs);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      float topv[kMaxK];
+      int tope[kMaxK];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        topv[j] = -FLT_MAX;
+        tope[j] = 0x7fffffff;
+      }
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
+        uint32_t v[32];
+        // up to four 8-column loads in flight per wait (warp-uniform bounds)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (c0 + 8 * j < p.n_pad) tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int e = c0 + i;
+          if (e < p.E) {
+            float cv = __uint_as_float(v[i]) + bf16_bits_to_float(__ldg(p.br + e));
+            int ce = e;
+            // insert into the sorted list: experts arrive in increasing index,
+            // so an equal logit never overtakes (lower index wins ties)
+            bool moved = false;
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+              if (j < p.k && (moved || cv > topv[j])) {
+                const float tv = topv[j];
+                const int te = tope[j];
+                topv[j] = cv;
+                tope[j] = ce;
+                cv = tv;
+                ce = te;
+                moved = true;
+              }
+            }
+          }
+        }
+      }
+      if (t < p.T) {
+        float ex[kMaxK], denom = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+          ex[j] = j < p.k ? __expf(topv[j] - topv[0]) : 0.f;
+          denom += ex[j];
+        }
+        const float inv = 1.0f / denom;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+          if (j < p.k) {
+            p.topk_idx[static_cast<int64_t>(t) * p.k + j] = tope[j];
+            p.topk_w[static_cast<int64_t>(t) * p.k + j] = ex[j] * inv;
+          }
+        }
+      }
+    } else if (lane == 0) {
+      record_status(p.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
     }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
-                         int32_t* topk_idx, float* topk_w, cudaStream_t s) {
-  dim3 grid((d.T + kTok - 1) / kTok);
-  if (d.E <= 16)
-    route_kernel<1><<<grid, kThreads, 0, s>>>(d.T, d.D, d.E, d.k, x, Wr, br, topk_idx, topk_w);
-  else if (d.E <= 32)
-    route_kernel<2><<<grid, kThreads, 0, s>>>(d.T, d.D, d.E, d.k, x, Wr, br, topk_idx, topk_w);
-  else if (d.E <= 64)
-    route_kernel<4><<<grid, kThreads, 0, s>>>(d.T, d.D, d.E, d.k, x, Wr, br, topk_idx, topk_w);
-  else if (d.E <= 128)
-    route_kernel<8><<<grid, kThreads, 0, s>>>(d.T, d.D, d.E, d.k, x, Wr, br, topk_idx, topk_w);
-  else
-    route_kernel<16><<<grid, kThreads, 0, s>>>(d.T, d.D, d.E, d.k, x, Wr, br, topk_idx, topk_w);
+                         int32_t* topk_idx, float* topk_w, int* status, cudaStream_t s) {
+  RouteParams p{};
+  p.T = d.T;
+  p.D = d.D;
+  p.E = d.E;
+  p.k = d.k;
+  p.n_pad = (d.E + 15) / 16 * 16;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.n_pad)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.br = br;
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.status = status;
+  CUtensorMap tx, tw;
+  if (!make_tmap_bf16(&tx, x, d.D, d.T, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tw, Wr, d.D, d.E, p.n_pad)) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + static_cast<size_t>(kStages) * (kABytes + p.n_pad * BK * 2) + 128;
+  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  route_tc_kernel<<<(d.T + BM - 1) / BM, kThreads, smem, s>>>(tx, tw, p);
   return cudaGetLastError();
 }
 

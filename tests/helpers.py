@@ -53,7 +53,7 @@ def run_stages(inp: synthetic.LayerInputs) -> GpuRun:
     h = torch.empty((R, s.I), dtype=torch.bfloat16, device=dev)
     o_perm = torch.empty((R, s.D), dtype=torch.float32, device=dev)
     y = torch.empty((s.T, s.D), dtype=torch.bfloat16, device=dev)
-    moe.moe_route(d, inp.x, inp.Wr, inp.br, topk_idx, topk_w)
+    moe.moe_route(d, inp.x, inp.Wr, inp.br, topk_idx, topk_w, ws)
     moe.moe_permute(d, topk_idx, counts, offsets, perm, inv, ws)
     moe.moe_gather(d, inp.x, perm, x_perm, ws)
     moe.moe_mlp1(d, x_perm, offsets, inp.W1, inp.b1, h, ws, W1_scales=inp.W1_scales)

@@ -60,8 +60,9 @@ def test_argument_errors_are_synchronous():
     d = moe.dims(64, 64, 4, 2, 64)
     vp = ctypes.c_void_p
     fake = vp(1 << 20)  # never dereferenced: validation fails first
-    assert lib.moe_route(d, None, fake, fake, fake, fake, None) == 1
-    assert lib.moe_route(d, vp((1 << 20) + 8), fake, fake, fake, fake, None) == 1  # misaligned x
+    assert lib.moe_route(d, None, fake, fake, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.moe_route(d, vp((1 << 20) + 8), fake, fake, fake, fake, fake, 1 << 30, None) == 1  # misaligned x
+    assert lib.moe_route(d, fake, fake, fake, fake, fake, fake, 16, None) == 3
     assert lib.moe_permute(d, fake, fake, fake, fake, fake, fake, 16, None) == 3  # workspace too small
     assert lib.moe_permute(d, fake, fake, fake, fake, fake, vp((1 << 20) + 4), 1 << 30, None) == 1
     w = _binding.Weight(None, None)

@@ -1,7 +1,10 @@
 """GPU parity of the CUDA path against the CPU oracle, through the C ABI.
 
 Bit-exact: expert indices, counts, offsets, perm, inv, gathered rows.
-Floating point: gate weights within 2e-6 absolute; layer output within
+Floating point: gate weights within 1e-5 absolute (the router logits are fp32
+tensor-core sums over D terms of size ~D^-1/2, off by a few 1e-6 from the
+fp64 ones; a logit error d moves a softmax weight w by at most 2*w*|d|, and
+__expf adds a few ulp); layer output within
 max|y - y_ref| <= 2e-2 * rms(y_ref) (bf16 weights) or 6e-2 (MXFP4), where
 y_ref is the oracle's output before its final bf16 rounding (two correct
 bf16 roundings of nearly equal values can land one ulp apart, and one ulp of
@@ -25,7 +28,7 @@ def _inputs(name, T=None, seed=None):
 def _check_routing(inp, run):
     _, idx_ref, w_ref = oracle.route(inp.x, inp.Wr, inp.br, inp.shape.k)
     assert torch.equal(run.topk_idx.cpu(), idx_ref)
-    assert float((run.topk_w.cpu() - w_ref).abs().max()) <= 2e-6
+    assert float((run.topk_w.cpu() - w_ref).abs().max()) <= 1e-5
     counts, offsets, perm, inv = oracle.permute(idx_ref, inp.shape.E)
     assert torch.equal(run.counts.cpu(), counts)
     assert torch.equal(run.offsets.cpu(), offsets)
