@@ -152,6 +152,25 @@ MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t
                          moe_weight_t W1, const uint16_t* b1, moe_weight_t W2, const uint16_t* b2,
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory -- e.g. code running where the memory budget is fixed up front by a
+ * host framework or serving runtime, or on a latency-critical path that must
+ * not call cudaMalloc (which can synchronise the device). This entry point
+ * has no counterpart in the layer's description; it is a deployment aid.
+ * Same arguments and outputs as moe_permute, minus ws: the per-block expert
+ * histogram it needs is kept in a fixed 256 KB array inside the library
+ * (held on every GPU that loads the library until the process exits), so it
+ * allocates nothing. Limit: ceil(T*k / 2048) * E <= 65536 (e.g. T*k <= 4M at
+ * E = 32, <= 512K at E = 256); larger sizes return MOE_ERR_UNSUPPORTED
+ * without enqueueing anything. The first call on each device looks up the
+ * array's device address with that device current; make that first call
+ * before any stream capture. Calls share the array, so two calls that overlap
+ * on the GPU (other streams or host threads) race. With no workspace there is
+ * no device status word: an out-of-range expert index shows up only as
+ * inv[a] = -1 and a missing count. */
+MOE_API moe_status_t moe_permute_noalloc(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                                 int32_t* perm, int32_t* inv, void* stream);
+
 /* Synchronise `stream`, return the device status recorded in ws since the
  * last read (MOE_OK if none) and clear it. */
 MOE_API moe_status_t moe_read_device_status(void* ws, void* stream);

@@ -22,7 +22,8 @@ STATUS = {
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_workspace_bytes", "moe_check_dims", "moe_route", "moe_permute", "moe_gather", "moe_mlp1", "moe_mlp2",
-           "moe_ffn_grouped", "moe_combine", "moe_forward", "moe_read_device_status", "moe_status_str")
+           "moe_ffn_grouped", "moe_combine", "moe_forward", "moe_read_device_status", "moe_status_str",
+           "moe_permute_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -68,6 +69,7 @@ def load(path: str = LIB_PATH):
         "moe_combine": (ctypes.c_int, [Dims, VP, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_forward": (ctypes.c_int, [Dims, VP, VP, VP, Weight, VP, Weight, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_read_device_status": (ctypes.c_int, [VP, VP]),
+        "moe_permute_noalloc": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP]),
         "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -154,6 +156,12 @@ def moe_combine(d, o_perm, inv, y, ws, stream=None):
 def moe_forward(d, x, Wr, br, W1, b1, W2, b2, y, ws, W1_scales=None, W2_scales=None, stream=None):
     _check(load().moe_forward(d, _p(x), _p(Wr), _p(br), _w(W1, W1_scales), _p(b1), _w(W2, W2_scales), _p(b2), _p(y),
                               _p(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_permute_noalloc(d, topk_idx, counts, offsets, perm, inv, stream=None):
+    """moe_permute without a workspace (scratch in a fixed library array)."""
+    _check(load().moe_permute_noalloc(d, _p(topk_idx), _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_read_device_status(ws, stream=None) -> int:

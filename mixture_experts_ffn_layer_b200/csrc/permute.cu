@@ -206,3 +206,64 @@ cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the permutation for callers that cannot allocate.
+//
+// The only scratch the permutation needs is the per-block expert histogram
+// (one int32 per (block of kPermChunk assignments, expert)). Here it lives in
+// a fixed array in the library's own device memory instead of a caller
+// workspace. Every GPU that loads the library holds this array until the
+// process exits. Calls share it: each call overwrites every entry it reads
+// (the histogram kernel writes all of its block's counts, so nothing has to
+// start at zero), and two calls whose kernels overlap on the GPU -- on two
+// streams, or on two host threads -- race on it.
+#include <mutex>
+
+namespace moe {
+namespace {
+
+// 65536 int32 = 256 KB: enough for ceil(T*k / 2048) * E <= 65536, e.g.
+// T*k <= 4M assignments at E = 32, or <= 512K at E = 256.
+constexpr int64_t kNoAllocScratchInts = int64_t(1) << 16;
+__device__ __align__(256) int32_t g_noalloc_block_counts[kNoAllocScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. The host-side
+// name of a __device__ array is only a stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+moe_status_t noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_block_counts) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status_t moe_permute_noalloc(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                                            int32_t* perm, int32_t* inv, void* stream) {
+  using namespace moe;
+  const moe_status_t dims_ok = moe_check_dims(d);
+  if (dims_ok != MOE_OK) return dims_ok;
+  if (!topk_idx || !counts || !offsets || !perm || !inv) return MOE_ERR_INVALID_ARG;
+  const int64_t R = static_cast<int64_t>(d.T) * d.k;
+  if (static_cast<int64_t>(perm_blocks(R)) * d.E > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;
+  int32_t* scratch = nullptr;
+  const moe_status_t st = noalloc_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  return launch_permute(d, topk_idx, counts, offsets, perm, inv, scratch, nullptr, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
