@@ -1,0 +1,109 @@
+"""Edge cases of the CUDA path against the oracle, through the C ABI:
+a single expert (a dense SwiGLU MLP), k = E, one token, empty experts, exact
+ties, the largest supported E and k, ragged tails, and device-side range
+errors reported through the status word without faulting."""
+import dataclasses
+
+import pytest
+import torch
+
+import mixture_experts_ffn_layer_b200 as moe
+import oracle
+import synthetic
+from helpers import TOL_BF16, assert_close_rms, run_stages
+
+pytestmark = pytest.mark.gpu
+
+BF16 = torch.bfloat16
+
+
+def _check_full(inp):
+    run = run_stages(inp)
+    assert run.status == 0, moe.status_str(run.status)
+    s = inp.shape
+    _, idx_ref, w_ref = oracle.route(inp.x, inp.Wr, inp.br, s.k)
+    assert torch.equal(run.topk_idx.cpu(), idx_ref)
+    assert float((run.topk_w.cpu() - w_ref).abs().max()) <= 1e-5
+    counts, offsets, perm, inv = oracle.permute(idx_ref, s.E)
+    for a, b in ((run.counts, counts), (run.offsets, offsets), (run.perm, perm), (run.inv, inv)):
+        assert torch.equal(a.cpu(), b)
+    _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, return_exact=True)
+    assert_close_rms(run.y, y_ref, TOL_BF16)
+    return run
+
+
+@pytest.mark.parametrize("T,D,E,k,I", [
+    (300, 64, 1, 1, 64),     # one expert: a dense SwiGLU MLP, ragged 300-row tail
+    (130, 128, 4, 4, 192),   # k = E: every token visits every expert
+    (1, 256, 8, 2, 128),     # one token
+    (517, 192, 256, 8, 64),  # largest supported E and k
+    (1000, 64, 3, 2, 320),   # non-power-of-two E, N tiles of 64 / 160
+])
+def test_shapes(T, D, E, k, I):
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", reject=oracle.gap_reject())
+    _check_full(inp)
+
+
+def test_empty_experts():
+    T, D, E, k, I = 200, 64, 16, 2, 64
+    base = synthetic.make_custom(T, D, E, k, I, seed=3)
+    # a strong bias on experts 3 and 11 leaves most experts with no rows
+    br = torch.full((E,), -8.0)
+    br[3] = br[11] = 8.0
+    br[7] = 0.0
+    br = br.to(BF16)
+    keep = ~oracle.gap_reject()(base.x, base.Wr, br, k)
+    x = base.x[keep].contiguous()
+    shape = synthetic.LayerShape("custom", x.shape[0], D, E, k, I)
+    inp = dataclasses.replace(base, shape=shape, x=x, br=br).to("cuda")
+    run = _check_full(inp)
+    assert int((run.counts == 0).sum()) >= 10
+
+
+def test_exact_ties_pick_lower_index():
+    T, D, E, k, I = 96, 64, 6, 3, 64
+    g = torch.Generator().manual_seed(5)
+    x = torch.randint(-2, 3, (T, D), generator=g).to(BF16)
+    base = torch.randint(-1, 2, (3, D), generator=g)
+    Wr = torch.cat([base, base]).to(BF16)  # experts e and e+3 tie exactly
+    inp = synthetic.make_custom(T, D, E, k, I, seed=6)
+    inp.x, inp.Wr, inp.br = x, Wr, torch.zeros(E, dtype=BF16)
+    inp = inp.to("cuda")
+    run = run_stages(inp)
+    _, idx_ref, _ = oracle.route(inp.x, inp.Wr, inp.br, k)
+    assert torch.equal(run.topk_idx.cpu(), idx_ref)
+    # ties are real: some token has an expert e and its twin e+3 both chosen, e first
+    pairs = [(r.index(e), r.index(e + 3)) for r in idx_ref.tolist() for e in range(3) if e in r and e + 3 in r]
+    assert pairs and all(a < b for a, b in pairs)
+
+
+def test_out_of_range_indices_are_reported_not_faulted():
+    T, E, k = 300, 8, 2
+    d = moe.dims(T, 64, E, k, 64)
+    ws = moe.alloc_workspace(d)
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32, device="cuda")
+    idx[5, 1] = E + 3
+    idx[77, 0] = -1
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    perm, inv = torch.empty(T * k, **i32), torch.empty(T * k, **i32)
+    moe.moe_permute(d, idx, counts, offsets, perm, inv, ws)
+    assert moe.moe_read_device_status(ws) == 6
+    assert moe.moe_read_device_status(ws) == 0  # read clears
+    assert int(inv[5 * k + 1]) == -1 and int(inv[77 * k]) == -1
+    assert int(offsets[-1]) == T * k - 2
+
+
+def test_bad_offsets_are_reported_and_skipped():
+    T, D, E, k, I = 256, 64, 4, 2, 64
+    R = T * k
+    d = moe.dims(T, D, E, k, I)
+    ws = moe.alloc_workspace(d)
+    x_perm = torch.zeros((R, D), dtype=BF16, device="cuda")
+    W1 = torch.zeros((E, 2 * I, D), dtype=BF16, device="cuda")
+    b1 = torch.zeros((E, 2 * I), dtype=BF16, device="cuda")
+    h = torch.full((R, I), 7.0, dtype=BF16, device="cuda")
+    offsets = torch.tensor([0, 100, 50, 400, R], dtype=torch.int32, device="cuda")  # not monotone
+    moe.moe_mlp1(d, x_perm, offsets, W1, b1, h, ws)
+    assert moe.moe_read_device_status(ws) == 6
+    assert bool((h == 7.0).all())  # nothing written
