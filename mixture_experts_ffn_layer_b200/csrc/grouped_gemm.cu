@@ -357,19 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c < p.n_tile) {
               float bv[8];
               unpack8(__ldg(reinterpret_cast<const uint4*>(bb + c)), bv);
-              float4 o0, o1;
-              o0.x = wgt * (__uint_as_float(v[8 * j + 0]) + bv[0]);
-              o0.y = wgt * (__uint_as_float(v[8 * j + 1]) + bv[1]);
-              o0.z = wgt * (__uint_as_float(v[8 * j + 2]) + bv[2]);
-              o0.w = wgt * (__uint_as_float(v[8 * j + 3]) + bv[3]);
-              o1.x = wgt * (__uint_as_float(v[8 * j + 4]) + bv[4]);
-              o1.y = wgt * (__uint_as_float(v[8 * j + 5]) + bv[5]);
-              o1.z = wgt * (__uint_as_float(v[8 * j + 6]) + bv[6]);
-              o1.w = wgt * (__uint_as_float(v[8 * j + 7]) + bv[7]);
-              if (valid) {
-                reinterpret_cast<float4*>(dst + c)[0] = o0;
-                reinterpret_cast<float4*>(dst + c)[1] = o1;
-              }
+              float ov[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) ov[i] = wgt * (__uint_as_float(v[8 * j + i]) + bv[i]);
+              // one 32-byte store: a full sector per thread (rows are 32-byte aligned)
+              if (valid) st_global_v8f(dst + c, ov);
             }
           }
         }

@@ -12,6 +12,7 @@
 // The combine (from-scratch GPT-OSS write-up, "weighted combination") is a
 // gather: every output row sums its k expert rows in slot order.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
@@ -103,75 +104,53 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_
   }
 }
 
-// x_perm[r, :] = x[perm[r] / k, :], one 16-byte vector per thread.
-__global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, uint4* __restrict__ x_perm,
-                                   int64_t R, int k, int T, int vec_per_row, int* status) {
-  const int64_t n = R * vec_per_row;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / vec_per_row;
-    const int c = static_cast<int>(i - r * vec_per_row);
-    const int32_t a = perm[r];
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (a >= 0 && a < R) {
-      v = x[static_cast<int64_t>(a / k) * vec_per_row + c];
-    } else if (c == 0) {
-      record_status(status, MOE_ERR_DEVICE_BOUNDS);
-    }
-    x_perm[i] = v;
-  }
+// x_perm[r, :] = x[perm[r] / k, :]. Grid (row, chunk block): each thread
+// copies one 32-byte vector (16 bf16) of one row.
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+                                   uint16_t* __restrict__ x_perm, int64_t R, int k, int D, int* status) {
+  const int64_t r = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= D / 16) return;
+  const int32_t a = perm[r];
+  uint32_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (a >= 0 && a < R)
+    sm100::ld_global_v8u(x + static_cast<int64_t>(a / k) * D + 16 * c, v);
+  else if (c == 0)
+    record_status(status, MOE_ERR_DEVICE_BOUNDS);
+  sm100::st_global_v8u(x_perm + r * D + 16 * c, v);
 }
 
-// y[t, :] = bf16( sum_j o_perm[inv[t*k + j], :] ), fp32 sum in slot order;
-// one thread per 8 outputs (two 16-byte fp32 loads per slot, one bf16 store).
-__global__ void combine_kernel(const float4* __restrict__ o_perm, const int32_t* __restrict__ inv,
-                               uint4* __restrict__ y, int T, int k, int64_t R, int vec_per_row, int* status) {
-  const int64_t n = static_cast<int64_t>(T) * vec_per_row;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / vec_per_row;
-    const int c = static_cast<int>(i - t * vec_per_row);
-    float acc[8];
+// y[t, :] = bf16( sum_j o_perm[inv[t*k + j], :] ), fp32 sum in slot order.
+// Grid (token, chunk block): each thread sums k 32-byte fp32 vectors and
+// stores 8 bf16.
+__global__ void combine_kernel(const float* __restrict__ o_perm, const int32_t* __restrict__ inv,
+                               uint16_t* __restrict__ y, int k, int64_t R, int D, int* status) {
+  const int64_t t = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= D / 8) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int j = 0; j < k; ++j) {
+    const int32_t r = __ldg(inv + t * k + j);
+    if (r < 0 || r >= R) {
+      if (c == 0) record_status(status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    float v[8];
+    sm100::ld_global_v8f(o_perm + static_cast<int64_t>(r) * D + 8 * c, v);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int32_t r = inv[t * k + j];
-      if (r < 0 || r >= R) {
-        if (c == 0) record_status(status, MOE_ERR_DEVICE_BOUNDS);
-        continue;
-      }
-      const float4* src = o_perm + (static_cast<int64_t>(r) * vec_per_row + c) * 2;
-      const float4 v0 = src[0], v1 = src[1];
-      acc[0] += v0.x;
-      acc[1] += v0.y;
-      acc[2] += v0.z;
-      acc[3] += v0.w;
-      acc[4] += v1.x;
-      acc[5] += v1.y;
-      acc[6] += v1.z;
-      acc[7] += v1.w;
-    }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    y[i] = out;
+    for (int q = 0; q < 8; ++q) acc[q] += v[q];
   }
+  uint4 out;
+  out.x = pack_bf16x2(acc[0], acc[1]);
+  out.y = pack_bf16x2(acc[2], acc[3]);
+  out.z = pack_bf16x2(acc[4], acc[5]);
+  out.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(y + t * D + 8 * c) = out;
 }
 
-int grid_for(int64_t n, int threads) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  int64_t blocks = (n + threads - 1) / threads;
-  int64_t cap = static_cast<int64_t>(sms) * 8;
-  return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
-}
+// Threads per block for n vectors per row: a multiple of 32, at most 256.
+int row_block(int n) { return n >= 256 ? 256 : (n + 31) / 32 * 32; }
+
 
 }  // namespace
 
@@ -187,21 +166,18 @@ cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm, int* status,
                           cudaStream_t s) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
-  const int vpr = d.D / 8;
-  const int threads = 256;
-  gather_rows_kernel<<<grid_for(R * vpr, threads), threads, 0, s>>>(reinterpret_cast<const uint4*>(x), perm,
-                                                                     reinterpret_cast<uint4*>(x_perm), R, d.k, d.T,
-                                                                     vpr, status);
+  const int n = d.D / 16, bs = row_block(n);
+  gather_rows_kernel<<<dim3(static_cast<unsigned>(R), (n + bs - 1) / bs), bs, 0, s>>>(x, perm, x_perm, R, d.k, d.D,
+                                                                                      status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32_t* inv, uint16_t* y, int* status,
                            cudaStream_t s) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
-  const int vpr = d.D / 8;
-  const int threads = 256;
-  combine_kernel<<<grid_for(static_cast<int64_t>(d.T) * vpr, threads), threads, 0, s>>>(
-      reinterpret_cast<const float4*>(o_perm), inv, reinterpret_cast<uint4*>(y), d.T, d.k, R, vpr, status);
+  const int n = d.D / 8, bs = row_block(n);
+  combine_kernel<<<dim3(static_cast<unsigned>(d.T), (n + bs - 1) / bs), bs, 0, s>>>(o_perm, inv, y, d.k, R, d.D,
+                                                                                    status);
   return cudaGetLastError();
 }
 
