@@ -34,6 +34,14 @@ sys.path.insert(0, ROOT)
 import synthetic  # noqa: E402
 
 WORKLOAD = "gptoss20b"
+WORKLOAD_NAMES = {
+    "gptoss20b": "gpt-oss-20b-shaped MoE FFN layer",
+    "gptoss120b_zipf": "gpt-oss-120b-shaped MoE FFN layer, skewed routing",
+    "gptoss20b_mxfp4": "gpt-oss-20b-shaped MoE FFN layer, MXFP4 expert weights",
+    "gptoss20b_mxfp4_decode": "gpt-oss-20b-shaped MoE FFN layer, MXFP4 expert weights, 64 tokens",
+    "debug": "debug-sized MoE FFN layer",
+    "tiny": "tiny MoE FFN layer",
+}
 METRIC = "MoE layer tokens/s and TFLOP/s at 1 B200, % of tensor-core peak"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -131,11 +139,13 @@ def run_ours(args):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    shape = synthetic.SHAPES[WORKLOAD]
-    inp = synthetic.make_inputs(WORKLOAD, seed=synthetic.SEEDS[WORKLOAD] + 1000 * rank, device=dev)
+    workload = args.workload
+    shape = synthetic.SHAPES[workload]
+    inp = synthetic.make_inputs(workload, seed=synthetic.SEEDS[workload] + 1000 * rank, device=dev)
     T, D, E, k, I = shape.T, shape.D, shape.E, shape.k, shape.I
     R = T * k
-    d = moe.dims(T, D, E, k, I)
+    mx = shape.wfmt == "mxfp4"
+    d = moe.dims(T, D, E, k, I, moe.MOE_W_MXFP4 if mx else moe.MOE_W_BF16)
     ws = moe.alloc_workspace(d, device=dev)
     i32 = dict(dtype=torch.int32, device=dev)
     topk_idx = torch.empty((T, k), **i32)
@@ -161,9 +171,9 @@ def run_ours(args):
         mark(2)
         moe.moe_gather(d, inp.x, perm, x_perm, ws)
         mark(3)
-        moe.moe_mlp1(d, x_perm, offsets, inp.W1, inp.b1, h, ws)
+        moe.moe_mlp1(d, x_perm, offsets, inp.W1, inp.b1, h, ws, W1_scales=inp.W1_scales)
         mark(4)
-        moe.moe_mlp2(d, h, perm, offsets, topk_w, inp.W2, inp.b2, o_perm, ws)
+        moe.moe_mlp2(d, h, perm, offsets, topk_w, inp.W2, inp.b2, o_perm, ws, W2_scales=inp.W2_scales)
         mark(5)
         moe.moe_combine(d, o_perm, inv, y, ws)
         mark(6)
@@ -204,7 +214,8 @@ def run_ours(args):
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        moe.moe_forward(d, x_dev, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws)
+        moe.moe_forward(d, x_dev, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws, W1_scales=inp.W1_scales,
+                        W2_scales=inp.W2_scales)
         y_host.copy_(y, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -236,12 +247,13 @@ def run_ours(args):
     peak_key = "bf16_tflops_sustained" if capped else "bf16_tflops"
     peak_tf = float(pk.get(peak_key, FALLBACK_PEAKS[peak_key]))
     mlp1_flops = 4.0 * R * D * I
+    wbytes = sum(t.numel() * t.element_size() for t in (inp.W1, inp.W2, inp.W1_scales, inp.W2_scales) if t is not None)
     mlp1_tf = mlp1_flops / (mlp1_ms / 1e3) / 1e12
     kernel_src = os.path.join(ROOT, "mixture_experts_ffn_layer_b200", "csrc", "grouped_gemm.cu")
     traffic = traffic_from_profile(kernel_src)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not mx:
         cpu = cpu_baseline(inp, budget_s=args.cpu_budget)
 
     if rank == 0:
@@ -249,9 +261,9 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights of the layer shape)",
-            "config": {"workload": "gpt-oss-20b-shaped MoE FFN layer", "T": T, "D": D, "E": E, "k": k, "I": I,
-                       "weights": "bf16", "tokens_per_gpu": T, "parallelism": f"replicas x{world} (token-sharded, "
-                       "no collective)", "l2": "inputs larger than L2 (expert weights 1.59 GB per step)"},
+            "config": {"workload": WORKLOAD_NAMES[workload], "T": T, "D": D, "E": E, "k": k, "I": I,
+                       "weights": shape.wfmt, "tokens_per_gpu": T, "parallelism": f"replicas x{world} (token-sharded, "
+                       "no collective)", "l2": f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB per step)"},
             "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peak_tf, "peak_kind": f"{peak_key} ({pk_kind})",
             "stages_ms": stage_ms,
             "roofline": {"kernel": "grouped mlp1 (tcgen05)", "bound": "tensor", "achieved": mlp1_tf, "peak": peak_tf,
@@ -259,7 +271,7 @@ def run_ours(args):
                          "algorithmic": f"4*R*D*I = {mlp1_flops:.4g} FLOP per launch"},
             "e2e": {"value": T * world / (e2e_ms / args.steps / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": (LAUNCHES_PER_STEP + (2 if mx else 0)) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -304,8 +316,8 @@ def run_reference(args):
         return
     import oracle
 
-    shape = synthetic.SHAPES[WORKLOAD]
-    inp = synthetic.make_inputs(WORKLOAD, seed=synthetic.SEEDS[WORKLOAD], device="cpu")
+    shape = synthetic.SHAPES[args.workload]
+    inp = synthetic.make_inputs(args.workload, seed=synthetic.SEEDS[args.workload], device="cpu")
     x, Wr, br = inp.x, inp.Wr, inp.br
     k, T = shape.k, shape.T
     per_step_s = max(1.0, args.ref_budget / max(1, args.steps + args.warmup))
@@ -316,7 +328,8 @@ def run_reference(args):
         xs = x[toks].contiguous()
         t0 = time.perf_counter()
         _, idx, w = oracle.route(xs, Wr, br, k)
-        oracle.ffn_tokens(xs, idx, w, inp.W1, inp.b1, inp.W2, inp.b2)
+        oracle.ffn_tokens(xs, idx, w, inp.W1, inp.b1, inp.W2, inp.b2, W1_scales=inp.W1_scales,
+                          W2_scales=inp.W2_scales)
         return time.perf_counter() - t0
 
     t1 = one(2, 0)
@@ -331,8 +344,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": "gpt-oss-20b-shaped MoE FFN layer", "T": T, "D": shape.D, "E": shape.E, "k": k,
-                   "I": shape.I, "weights": "bf16"},
+        "config": {"workload": WORKLOAD_NAMES[args.workload], "T": T, "D": shape.D, "E": shape.E, "k": k,
+                   "I": shape.I, "weights": shape.wfmt},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"{n} of {T} tokens per step (route + FFN + combine per token)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -346,6 +359,8 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_NAMES), default=WORKLOAD,
+                    help="the bench line is the 20B shape; the others are for inspection")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
