@@ -21,8 +21,8 @@
  *
  * Conventions for every entry point:
  *  - All pointers are DEVICE pointers unless stated otherwise; every tensor
- *    is dense, row-major, and at least 16-byte aligned. bf16 tensors are
- *    passed as uint16_t bit patterns.
+ *    is dense, row-major, and at least 32-byte aligned (a misaligned pointer
+ *    is an argument error). bf16 tensors are passed as uint16_t bit patterns.
  *  - The caller owns every buffer and the stream. The library allocates
  *    nothing; scratch lives in the caller's workspace `ws` of `ws_bytes`
  *    bytes (at least moe_workspace_bytes(d)), zero-filled once before its
@@ -56,7 +56,7 @@ extern "C" {
 
 typedef enum {
   MOE_OK = 0,
-  MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, k > E, misaligned pointer */
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, k > E, pointer not 32-byte aligned */
   MOE_ERR_UNSUPPORTED = 2,   /* sizes outside the supported set above */
   MOE_ERR_WORKSPACE = 3,     /* ws_bytes < moe_workspace_bytes(d) */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, tensor map) */
@@ -119,7 +119,10 @@ MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* 
  * for r in [offsets[e], offsets[e+1]):
  *   u = W1[e] . x_perm[r] + b1[e] (fp32 accumulate), h[r,i] = bf16(silu(u[i]) * u[I+i]).
  *   x_perm (R,D) bf16, offsets (E+1), W1 (E,2I,D), b1 (E,2I) bf16 -> h (R,I) bf16.
- * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile). */
+ * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile).
+ * MXFP4 weights: with T*k <= 16*E (a few rows per expert) the codes are
+ * decoded in registers by a weight-streaming kernel; otherwise they are
+ * expanded to bf16 in ws first (exact) and the bf16 GEMM runs. */
 MOE_API moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
                       const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream);
 

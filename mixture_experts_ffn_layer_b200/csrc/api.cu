@@ -40,7 +40,9 @@ WsLayout ws_layout(const moe_dims_t& d) {
   return L;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Every tensor must be 32-byte aligned: the memory-bound kernels move 32-byte
+// vectors and TMA needs 16.
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <class T>
 T* at(void* ws, size_t off) {
@@ -50,13 +52,13 @@ T* at(void* ws, size_t off) {
 int* status_word(void* ws) { return static_cast<int*>(ws); }
 
 moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes) {
-  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned32(ws)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < ws_layout(d).total) return MOE_ERR_WORKSPACE;
   return MOE_OK;
 }
 
 moe_status_t check_weight(const moe_dims_t& d, const moe_weight_t& w) {
-  if (!w.data || !aligned16(w.data)) return MOE_ERR_INVALID_ARG;
+  if (!w.data || !aligned32(w.data)) return MOE_ERR_INVALID_ARG;
   if (d.wfmt == MOE_W_MXFP4 && (!w.scales)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
@@ -113,7 +115,7 @@ moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, cons
                        float* topk_w, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
   MOE_REQUIRE(x && Wr && br && topk_idx && topk_w);
-  MOE_REQUIRE(aligned16(x) && aligned16(Wr));
+  MOE_REQUIRE(aligned32(x) && aligned32(Wr));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   return cuda_status(
       launch_route(d, x, Wr, br, topk_idx, topk_w, status_word(ws), static_cast<cudaStream_t>(stream)));
@@ -132,7 +134,7 @@ moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts,
 moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm, void* ws,
                         size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
-  MOE_REQUIRE(x && perm && x_perm && aligned16(x) && aligned16(x_perm));
+  MOE_REQUIRE(x && perm && x_perm && aligned32(x) && aligned32(x_perm));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   return cuda_status(launch_gather(d, x, perm, x_perm, status_word(ws), static_cast<cudaStream_t>(stream)));
 }
@@ -140,10 +142,13 @@ moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* perm, ui
 moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
                       const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
-  MOE_REQUIRE(x_perm && offsets && b1 && h && aligned16(x_perm) && aligned16(b1) && aligned16(h));
+  MOE_REQUIRE(x_perm && offsets && b1 && h && aligned32(x_perm) && aligned32(b1) && aligned32(h));
   MOE_TRY(check_weight(d, W1));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (skinny_fp4_applies(d))
+    return launch_mlp1_fp4_skinny(d, x_perm, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h,
+                                  status_word(ws), s);
   const WsLayout L = ws_layout(d);
   const uint16_t* w1 = nullptr;
   MOE_TRY(weight_bf16(d, W1, 2 * static_cast<int64_t>(d.I), d.D, ws, L.w1_deq, s, &w1));
@@ -154,10 +159,13 @@ moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, cons
                       const float* topk_w, moe_weight_t W2, const uint16_t* b2, float* o_perm, void* ws,
                       size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
-  MOE_REQUIRE(h && perm && offsets && topk_w && b2 && o_perm && aligned16(h) && aligned16(b2) && aligned16(o_perm));
+  MOE_REQUIRE(h && perm && offsets && topk_w && b2 && o_perm && aligned32(h) && aligned32(b2) && aligned32(o_perm));
   MOE_TRY(check_weight(d, W2));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (skinny_fp4_applies(d))
+    return launch_mlp2_fp4_skinny(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
+                                  o_perm, status_word(ws), s);
   const WsLayout L = ws_layout(d);
   const uint16_t* w2 = nullptr;
   MOE_TRY(weight_bf16(d, W2, d.D, d.I, ws, L.w2_deq, s, &w2));
@@ -181,7 +189,7 @@ moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* per
 moe_status_t moe_combine(moe_dims_t d, const float* o_perm, const int32_t* inv, uint16_t* y, void* ws,
                          size_t ws_bytes, void* stream) {
   MOE_TRY(moe_check_dims(d));
-  MOE_REQUIRE(o_perm && inv && y && aligned16(o_perm) && aligned16(y));
+  MOE_REQUIRE(o_perm && inv && y && aligned32(o_perm) && aligned32(y));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   return cuda_status(launch_combine(d, o_perm, inv, y, status_word(ws), static_cast<cudaStream_t>(stream)));
 }

@@ -9,6 +9,7 @@
 // so this expansion loses nothing and the bf16 tensor-core GEMMs then compute
 // the MXFP4 layer exactly as they compute the bf16 one.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
@@ -25,26 +26,26 @@ __device__ __forceinline__ float e8m0_value(uint32_t s) {
   return __uint_as_float(s << 23);
 }
 
-// One thread expands 8 consecutive elements (4 code bytes, one scale).
-__global__ void dequant_mxfp4_kernel(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                     uint4* __restrict__ out, int64_t n8) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+// One thread expands 16 consecutive elements (8 code bytes, one scale) into
+// one 32-byte store.
+__global__ void dequant_mxfp4_kernel(const uint2* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                     uint16_t* __restrict__ out, int64_t n16) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t w = codes[i];
-    const float sc = e8m0_value(scales[i >> 2]);  // 8 elements per thread, 32 per scale
-    float v[8];
+    const uint2 w2 = __ldg(codes + i);
+    const float sc = e8m0_value(__ldg(scales + (i >> 1)));  // 16 elements per thread, 32 per scale
+    uint32_t packed[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint32_t c = (w >> (4 * q)) & 0xfu;
-      const float mag = e2m1_magnitude(c) * sc;
-      v[q] = (c & 8u) ? -mag : mag;
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w = h ? w2.y : w2.x;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t c0 = (w >> (8 * q)) & 0xfu, c1 = (w >> (8 * q + 4)) & 0xfu;
+        const float m0 = e2m1_magnitude(c0) * sc, m1 = e2m1_magnitude(c1) * sc;
+        packed[4 * h + q] = pack_bf16x2((c0 & 8u) ? -m0 : m0, (c1 & 8u) ? -m1 : m1);
+      }
     }
-    uint4 o;
-    o.x = pack_bf16x2(v[0], v[1]);
-    o.y = pack_bf16x2(v[2], v[3]);
-    o.z = pack_bf16x2(v[4], v[5]);
-    o.w = pack_bf16x2(v[6], v[7]);
-    out[i] = o;
+    sm100::st_global_v8u(out + 16 * i, packed);
   }
 }
 
@@ -52,16 +53,16 @@ __global__ void dequant_mxfp4_kernel(const uint32_t* __restrict__ codes, const u
 
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t E, int64_t N, int64_t K,
                                  uint16_t* out, cudaStream_t s) {
-  const int64_t n8 = E * N * K / 8;
+  const int64_t n16 = E * N * K / 16;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int threads = 256;
-  int64_t blocks = (n8 + threads - 1) / threads;
+  int64_t blocks = (n16 + threads - 1) / threads;
   if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
   if (blocks < 1) blocks = 1;
-  dequant_mxfp4_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(reinterpret_cast<const uint32_t*>(codes), scales,
-                                                                     reinterpret_cast<uint4*>(out), n8);
+  dequant_mxfp4_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales,
+                                                                     out, n16);
   return cudaGetLastError();
 }
 
