@@ -10,7 +10,8 @@ namespace moe {
 namespace {
 
 struct WsLayout {
-  size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, w1_deq, w2_deq, total;
+  size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, w1_deq, w2_deq, tok16,
+      total;
 };
 
 WsLayout ws_layout(const moe_dims_t& d) {
@@ -32,7 +33,10 @@ WsLayout ws_layout(const moe_dims_t& d) {
   L.x_perm = take(static_cast<size_t>(R) * d.D * 2);
   L.h = take(static_cast<size_t>(R) * d.I * 2);
   L.o_perm = take(static_cast<size_t>(R) * d.D * 4);
-  if (d.wfmt == MOE_W_MXFP4) {
+  if (skinny_fp4_applies(d)) {
+    // routed rows (x_perm, then h) in f16 for the weight-streaming MXFP4 kernels
+    L.tok16 = take(static_cast<size_t>(R) * (d.D > d.I ? d.D : d.I) * 2);
+  } else if (d.wfmt == MOE_W_MXFP4) {
     L.w1_deq = take(static_cast<size_t>(d.E) * 2 * d.I * d.D * 2);
     L.w2_deq = take(static_cast<size_t>(d.E) * d.D * d.I * 2);
   }
@@ -146,10 +150,10 @@ moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offse
   MOE_TRY(check_weight(d, W1));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(d);
   if (skinny_fp4_applies(d))
     return launch_mlp1_fp4_skinny(d, x_perm, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h,
-                                  status_word(ws), s);
-  const WsLayout L = ws_layout(d);
+                                  at<uint16_t>(ws, L.tok16), status_word(ws), s);
   const uint16_t* w1 = nullptr;
   MOE_TRY(weight_bf16(d, W1, 2 * static_cast<int64_t>(d.I), d.D, ws, L.w1_deq, s, &w1));
   return launch_mlp1(d, x_perm, offsets, w1, b1, h, status_word(ws), s);
@@ -163,10 +167,10 @@ moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, cons
   MOE_TRY(check_weight(d, W2));
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(d);
   if (skinny_fp4_applies(d))
     return launch_mlp2_fp4_skinny(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
-                                  o_perm, status_word(ws), s);
-  const WsLayout L = ws_layout(d);
+                                  o_perm, at<uint16_t>(ws, L.tok16), status_word(ws), s);
   const uint16_t* w2 = nullptr;
   MOE_TRY(weight_bf16(d, W2, d.D, d.I, ws, L.w2_deq, s, &w2));
   return launch_mlp2(d, h, perm, offsets, topk_w, w2, b2, o_perm, status_word(ws), s);

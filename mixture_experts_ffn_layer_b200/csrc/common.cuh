@@ -65,11 +65,11 @@ moe_status_t launch_mlp2(const moe_dims_t& d, const uint16_t* h, const int32_t* 
 bool skinny_fp4_applies(const moe_dims_t& d);
 moe_status_t launch_mlp1_fp4_skinny(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
                                     const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                                    int* status, cudaStream_t s);
+                                    uint16_t* tok16, int* status, cudaStream_t s);
 moe_status_t launch_mlp2_fp4_skinny(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
                                     const int32_t* offsets, const float* topk_w, const uint8_t* codes,
-                                    const uint8_t* scales, const uint16_t* b2, float* o_perm, int* status,
-                                    cudaStream_t s);
+                                    const uint8_t* scales, const uint16_t* b2, float* o_perm, uint16_t* tok16,
+                                    int* status, cudaStream_t s);
 
 // MXFP4 -> bf16 expansion of an (E, N, K) expert weight (mxfp4.cu).
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t E, int64_t N, int64_t K,
