@@ -126,6 +126,24 @@ def traffic_from_profile(kernel_src: str):
         return None
 
 
+def max_over_ranks(times_ms, world, device="cpu"):
+    """Element-wise max of per-rank CUDA-event times (the slowest rank sets
+    the step time); identity on one rank."""
+    t = torch.tensor(times_ms, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def step_throughput(elapsed_ms, steps, tokens_per_rank, world):
+    """(ms per step, whole-job tokens/s): every rank processes its own batch of
+    tokens_per_rank tokens per step (replicas, weak scaling)."""
+    ms = elapsed_ms / steps
+    return ms, tokens_per_rank * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import mixture_experts_ffn_layer_b200 as moe
@@ -229,15 +247,9 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([elapsed_ms, e2e_ms, stage_ms["mlp1"]], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, mlp1_ms = times.tolist()
-    ms_per_step = elapsed_ms / args.steps
+    elapsed_ms, e2e_ms, mlp1_ms = max_over_ranks([elapsed_ms, e2e_ms, stage_ms["mlp1"]], world, dev)
+    ms_per_step, value = step_throughput(elapsed_ms, args.steps, T, world)
     tokens_total = T * world
-    value = tokens_total / (ms_per_step / 1e3)
     tflops = shape.flops * world / (ms_per_step / 1e3) / 1e12
 
     pk, pk_kind = peaks()

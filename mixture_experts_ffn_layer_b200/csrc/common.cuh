@@ -37,17 +37,21 @@ struct Launch {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Permutation block size: assignments per histogram/scatter block.
-constexpr int kPermChunk = 2048;
+// Permutation: assignments per histogram/scatter block (a multiple of the
+// block size), and the larger chunk of the workspace-free variant (its fixed
+// histogram array bounds ceil(T*k / chunk) * E).
+constexpr int kPermChunk = 512;
+constexpr int kPermChunkNoAlloc = 2048;
 constexpr int kPermThreads = 256;
 
-inline int perm_blocks(int64_t R) { return static_cast<int>((R + kPermChunk - 1) / kPermChunk); }
+inline int perm_blocks(int64_t R, int chunk = kPermChunk) { return static_cast<int>((R + chunk - 1) / chunk); }
 
 // Kernel launchers (defined in the .cu files).
 cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
                          int32_t* topk_idx, float* topk_w, int* status, cudaStream_t s);
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
-                           int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s);
+                           int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
+                           int chunk = kPermChunk);
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
                           int* status, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32_t* inv, uint16_t* y,
@@ -59,6 +63,13 @@ moe_status_t launch_mlp1(const moe_dims_t& d, const uint16_t* x_perm, const int3
 moe_status_t launch_mlp2(const moe_dims_t& d, const uint16_t* h, const int32_t* perm, const int32_t* offsets,
                          const float* topk_w, const uint16_t* W2, const uint16_t* b2, float* o_perm,
                          int* status, cudaStream_t s);
+
+// The same GEMMs on SM pairs, 256-row tiles (grouped_gemm_pair.cu).
+moe_status_t launch_mlp1_pair(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
+                              const uint16_t* W1, const uint16_t* b1, uint16_t* h, int* status, cudaStream_t s);
+moe_status_t launch_mlp2_pair(const moe_dims_t& d, const uint16_t* h, const int32_t* perm, const int32_t* offsets,
+                              const float* topk_w, const uint16_t* W2, const uint16_t* b2, float* o_perm,
+                              int* status, cudaStream_t s);
 
 // MXFP4 weights with few routed rows per expert (skinny_fp4.cu): the codes
 // are decoded in registers; no expansion pass.

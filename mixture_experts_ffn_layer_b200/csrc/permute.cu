@@ -4,7 +4,7 @@
 // grouped GEMMs with rows sorted by expert and offsets = cumsum of
 // num_tokens_per_expert, computed without a device-to-host sync. Here the
 // R = T*k assignments a = t*k + j are sorted stably by expert in two launches:
-//   1. per-block histograms of kPermChunk assignments (shared-memory counters);
+//   1. per-block histograms of `chunk` assignments (shared-memory counters);
 //   2. each block derives its per-expert base from the histograms of the
 //      blocks before it plus the exclusive scan over experts, then ranks its
 //      assignments in order with warp match/popc and per-warp counts -- the
@@ -18,12 +18,13 @@ namespace moe {
 namespace {
 
 __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
-                                                                 int32_t* __restrict__ block_counts, int* status) {
+                                                                 int chunk, int32_t* __restrict__ block_counts,
+                                                                 int* status) {
   __shared__ int cnt[256];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  const int64_t a0 = static_cast<int64_t>(blockIdx.x) * kPermChunk;
-  const int64_t a1 = min(a0 + kPermChunk, R);
+  const int64_t a0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t a1 = min(a0 + chunk, R);
   for (int64_t a = a0 + threadIdx.x; a < a1; a += blockDim.x) {
     int e = idx[a];
     if (e >= 0 && e < E)
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* 
 }
 
 __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
-                                                                    const int32_t* __restrict__ block_counts,
+                                                                    int chunk, const int32_t* __restrict__ block_counts,
                                                                     int32_t* __restrict__ counts,
                                                                     int32_t* __restrict__ offsets,
                                                                     int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
@@ -71,9 +72,9 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_
   }
   __syncthreads();
 
-  const int64_t a0 = static_cast<int64_t>(blk) * kPermChunk;
+  const int64_t a0 = static_cast<int64_t>(blk) * chunk;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int sub = 0; sub < kPermChunk; sub += kPermThreads) {
+  for (int sub = 0; sub < chunk; sub += kPermThreads) {
     for (int i = tid; i < kWarps * 256; i += kPermThreads) (&wcnt[0][0])[i] = 0;
     __syncthreads();
     const int64_t a = a0 + sub + tid;
@@ -155,11 +156,13 @@ int row_block(int n) { return n >= 256 ? 256 : (n + 31) / 32 * 32; }
 }  // namespace
 
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
-                           int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s) {
+                           int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
+                           int chunk) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
-  const int nblk = perm_blocks(R);
-  perm_hist_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, block_counts, status);
-  perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, block_counts, counts, offsets, perm, inv);
+  const int nblk = static_cast<int>((R + chunk - 1) / chunk);
+  perm_hist_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, chunk, block_counts, status);
+  perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, chunk, block_counts, counts, offsets, perm,
+                                                    inv);
   return cudaGetLastError();
 }
 
@@ -187,7 +190,7 @@ cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32
 // moe_permute_noalloc: the permutation for callers that cannot allocate.
 //
 // The only scratch the permutation needs is the per-block expert histogram
-// (one int32 per (block of kPermChunk assignments, expert)). Here it lives in
+// (one int32 per (block of kPermChunkNoAlloc = 2048 assignments, expert)). Here it lives in
 // a fixed array in the library's own device memory instead of a caller
 // workspace. Every GPU that loads the library holds this array until the
 // process exits. Calls share it: each call overwrites every entry it reads
@@ -234,12 +237,12 @@ extern "C" moe_status_t moe_permute_noalloc(moe_dims_t d, const int32_t* topk_id
   if (dims_ok != MOE_OK) return dims_ok;
   if (!topk_idx || !counts || !offsets || !perm || !inv) return MOE_ERR_INVALID_ARG;
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
-  if (static_cast<int64_t>(perm_blocks(R)) * d.E > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(perm_blocks(R, kPermChunkNoAlloc)) * d.E > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;
   int32_t* scratch = nullptr;
   const moe_status_t st = noalloc_scratch(&scratch);
   if (st != MOE_OK) return st;
-  return launch_permute(d, topk_idx, counts, offsets, perm, inv, scratch, nullptr, static_cast<cudaStream_t>(stream)) ==
-                 cudaSuccess
+  return launch_permute(d, topk_idx, counts, offsets, perm, inv, scratch, nullptr, static_cast<cudaStream_t>(stream),
+                        kPermChunkNoAlloc) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

@@ -8,7 +8,7 @@
 // The logits are a dense contraction (T x D) . (D x E), so each CTA computes a
 // 128-token tile of them with tcgen05.mma (M=128, N=E rounded up to 16, K=D)
 // into TMEM, fed by TMA (x rows and all of Wr, 64-wide K slices, 128-byte
-// swizzle, 4-stage ring). Its epilogue is one thread per token (= TMEM lane):
+// swizzle, a ring as deep as shared memory allows: only T/128 CTAs stream x). Its epilogue is one thread per token (= TMEM lane):
 // it streams the token's E logits out of TMEM, adds the bias, keeps a sorted
 // top-k in registers and writes the normalised gate weights. x is read once
 // from HBM; Wr stays L2-resident.
@@ -23,13 +23,14 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BK = 64, kStages = 4, kThreads = 192, kMaxK = 8;
+constexpr int BM = 128, BK = 64, kMaxStages = 12, kThreads = 192, kMaxK = 8;
 constexpr int kABytes = BM * BK * 2;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 struct RouteParams {
   int T, D, E, k;
   int n_pad;        // MMA N: E rounded up to a multiple of 16
+  int stages;       // TMA ring depth (as many as fit: few CTAs stream all of x)
   uint32_t tmem_cols;
   const uint16_t* br;
   int32_t* topk_idx;
@@ -43,17 +44,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t stage_bytes = kABytes + p.n_pad * BK * 2;
+  const int kStages = p.stages;
   uint8_t* ctrl = smem + kStages * stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);  // full[S] empty[S] tfull done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * kStages + 2));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * kMaxStages + 2));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  const uint32_t tfull_bar = bar0 + 8u * (2 * kStages);
-  const uint32_t done_bar = bar0 + 8u * (2 * kStages + 1);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * kMaxStages);
+  const uint32_t done_bar = bar0 + 8u * (2 * kMaxStages + 1);
   const int t0 = blockIdx.x * BM;
   const int KB = (p.D + BK - 1) / BK;
 
@@ -244,7 +246,10 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
   CUtensorMap tx, tw;
   if (!make_tmap_bf16(&tx, x, d.D, d.T, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tw, Wr, d.D, d.E, p.n_pad)) return cudaErrorInvalidValue;
-  const size_t smem = 1024 + static_cast<size_t>(kStages) * (kABytes + p.n_pad * BK * 2) + 128;
+  const size_t stage_bytes = kABytes + static_cast<size_t>(p.n_pad) * BK * 2;
+  p.stages = static_cast<int>((200 * 1024) / stage_bytes);
+  if (p.stages > kMaxStages) p.stages = kMaxStages;
+  const size_t smem = 1024 + p.stages * stage_bytes + 8 * (2 * kMaxStages + 2) + 16;
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -38,6 +38,8 @@ def _check_full(inp):
     (1, 256, 8, 2, 128),     # one token
     (517, 192, 256, 8, 64),  # largest supported E and k
     (1000, 64, 3, 2, 320),   # non-power-of-two E, N tiles of 64 / 160
+    (4200, 128, 4, 2, 192),  # >= 2048 rows per expert: SM-pair (256-row) GEMM tiles
+    (8500, 64, 2, 1, 128),   # pair tiles, ragged segments
 ])
 def test_shapes(T, D, E, k, I):
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", reject=oracle.gap_reject())
