@@ -178,6 +178,13 @@ MOE_API moe_status_t moe_permute_noalloc(moe_dims_t d, const int32_t* topk_idx, 
  * last read (MOE_OK if none) and clear it. */
 MOE_API moe_status_t moe_read_device_status(void* ws, void* stream);
 
+/* Self-test of the device-side failure detection: enqueue a one-thread
+ * kernel that waits on an mbarrier nothing will arrive on, using the same
+ * bounded wait as every tcgen05 kernel, gives up after limit_ns (at most 2 s)
+ * and records MOE_ERR_TIMEOUT in ws's status word. Read it with
+ * moe_read_device_status(); the context stays usable. */
+MOE_API moe_status_t moe_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_str(moe_status_t s);
 

@@ -14,7 +14,7 @@ import torch
 from ._binding import (  # noqa: F401
     MOE_W_BF16, MOE_W_MXFP4, EXPORTS, MoeError, Dims, dims, load, workspace_bytes, alloc_workspace, check_dims,
     moe_route, moe_permute, moe_gather, moe_mlp1, moe_mlp2, moe_ffn_grouped, moe_combine, moe_forward,
-    moe_read_device_status, status_str, moe_permute_noalloc,
+    moe_read_device_status, status_str, moe_permute_noalloc, moe_selftest_wait_timeout,
 )
 
 

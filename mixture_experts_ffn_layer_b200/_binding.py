@@ -23,7 +23,7 @@ STATUS = {
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_workspace_bytes", "moe_check_dims", "moe_route", "moe_permute", "moe_gather", "moe_mlp1", "moe_mlp2",
            "moe_ffn_grouped", "moe_combine", "moe_forward", "moe_read_device_status", "moe_status_str",
-           "moe_permute_noalloc")
+           "moe_permute_noalloc", "moe_selftest_wait_timeout")
 
 
 class MoeError(RuntimeError):
@@ -70,6 +70,7 @@ def load(path: str = LIB_PATH):
         "moe_forward": (ctypes.c_int, [Dims, VP, VP, VP, Weight, VP, Weight, VP, VP, VP, ctypes.c_size_t, VP]),
         "moe_read_device_status": (ctypes.c_int, [VP, VP]),
         "moe_permute_noalloc": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP]),
+        "moe_selftest_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
         "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -162,6 +163,10 @@ def moe_permute_noalloc(d, topk_idx, counts, offsets, perm, inv, stream=None):
     """moe_permute without a workspace (scratch in a fixed library array)."""
     _check(load().moe_permute_noalloc(d, _p(topk_idx), _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)),
            "moe_permute_noalloc")
+
+
+def moe_selftest_wait_timeout(ws, limit_ns: int, stream=None):
+    _check(load().moe_selftest_wait_timeout(_p(ws), limit_ns, _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def moe_read_device_status(ws, stream=None) -> int:

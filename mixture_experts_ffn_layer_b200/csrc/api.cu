@@ -254,3 +254,32 @@ const char* moe_status_str(moe_status_t s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded wait every tcgen05 kernel uses: one thread waits on
+// an mbarrier that nothing will arrive on, gives up after limit_ns and
+// records MOE_ERR_TIMEOUT in the status word, exactly as a stalled pipeline
+// would. The context stays usable.
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+__global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = sm100::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    sm100::fence_mbar_init();
+    if (!sm100::mbar_wait_bounded(b, 0, nullptr, limit_ns)) record_status(status, MOE_ERR_TIMEOUT);
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status_t moe_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream) {
+  if (!ws || limit_ns == 0 || limit_ns > 2000000000ull) return MOE_ERR_INVALID_ARG;
+  moe::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int*>(ws), limit_ns);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

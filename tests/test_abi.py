@@ -72,4 +72,7 @@ def test_argument_errors_are_synchronous():
     assert lib.moe_mlp1(dq, fake, fake, wq, fake, fake, fake, 1 << 30, None) == 1
     assert lib.moe_forward(moe.dims(64, 64, 4, 9, 64), fake, fake, fake, w, fake, w, fake, fake, fake, 0, None) == 1
     assert lib.moe_read_device_status(None, None) == 1
+    assert lib.moe_selftest_wait_timeout(None, 1000, None) == 1
+    assert lib.moe_selftest_wait_timeout(fake, 0, None) == 1
+    assert lib.moe_selftest_wait_timeout(fake, 3_000_000_000, None) == 1
     assert moe.status_str(6) == "device: index or offset out of range"

@@ -109,3 +109,19 @@ def test_bad_offsets_are_reported_and_skipped():
     moe.moe_mlp1(d, x_perm, offsets, W1, b1, h, ws)
     assert moe.moe_read_device_status(ws) == 6
     assert bool((h == 7.0).all())  # nothing written
+
+
+def test_bounded_wait_times_out_and_reports():
+    # a wait on an mbarrier nothing arrives on gives up after 20 ms and reports
+    # MOE_ERR_TIMEOUT; the context stays usable afterwards
+    import time
+
+    d = moe.dims(64, 64, 4, 2, 64)
+    ws = moe.alloc_workspace(d)
+    t0 = time.perf_counter()
+    moe.moe_selftest_wait_timeout(ws, 20_000_000)
+    assert moe.moe_read_device_status(ws) == 5
+    assert 0.015 < time.perf_counter() - t0 < 1.5
+    assert moe.moe_read_device_status(ws) == 0
+    inp = synthetic.make_inputs("tiny", device="cuda", reject=oracle.gap_reject())
+    assert run_stages(inp).status == 0
