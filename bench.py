@@ -21,6 +21,7 @@ import hashlib
 import io
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -125,9 +126,9 @@ def traffic_from_profile():
         return None
     fields = {}
     for line in open(p):
-        if ":" in line and line.startswith("- "):
-            k, v = line[2:].split(":", 1)
-            fields[k.strip()] = v.strip().strip("`")
+        m = re.match(r"- (\w+): `([^`]*)`", line)
+        if m:
+            fields[m.group(1)] = m.group(2)
     if fields.get("kernel_sources_sha256_16") != gemm_source_hash():
         return None
     try:

@@ -33,7 +33,7 @@ WsLayout ws_layout(const moe_dims_t& d) {
   L.x_perm = take(static_cast<size_t>(R) * d.D * 2);
   L.h = take(static_cast<size_t>(R) * d.I * 2);
   L.o_perm = take(static_cast<size_t>(R) * d.D * 4);
-  if (skinny_fp4_applies(d)) {
+  if (stream_fp4_applies(d)) {
     // routed rows (x_perm, then h) in f16 for the weight-streaming MXFP4 kernels
     L.tok16 = take(static_cast<size_t>(R) * (d.D > d.I ? d.D : d.I) * 2);
   } else if (d.wfmt == MOE_W_MXFP4) {
@@ -63,7 +63,7 @@ moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes) {
 
 moe_status_t check_weight(const moe_dims_t& d, const moe_weight_t& w) {
   if (!w.data || !aligned32(w.data)) return MOE_ERR_INVALID_ARG;
-  if (d.wfmt == MOE_W_MXFP4 && (!w.scales)) return MOE_ERR_INVALID_ARG;
+  if (d.wfmt == MOE_W_MXFP4 && (!w.scales || !aligned32(w.scales))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -157,8 +157,8 @@ moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offse
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(d);
-  if (skinny_fp4_applies(d))
-    return launch_mlp1_fp4_skinny(d, x_perm, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h,
+  if (stream_fp4_applies(d))
+    return launch_mlp1_fp4_stream(d, x_perm, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h,
                                   at<uint16_t>(ws, L.tok16), status_word(ws), s);
   const uint16_t* w1 = nullptr;
   MOE_TRY(weight_bf16(d, W1, 2 * static_cast<int64_t>(d.I), d.D, ws, L.w1_deq, s, &w1));
@@ -175,8 +175,8 @@ moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, cons
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(d);
-  if (skinny_fp4_applies(d))
-    return launch_mlp2_fp4_skinny(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
+  if (stream_fp4_applies(d))
+    return launch_mlp2_fp4_stream(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
                                   o_perm, at<uint16_t>(ws, L.tok16), status_word(ws), s);
   const uint16_t* w2 = nullptr;
   MOE_TRY(weight_bf16(d, W2, d.D, d.I, ws, L.w2_deq, s, &w2));

@@ -71,13 +71,14 @@ moe_status_t launch_mlp2_pair(const moe_dims_t& d, const uint16_t* h, const int3
                               const float* topk_w, const uint16_t* W2, const uint16_t* b2, float* o_perm,
                               int* status, cudaStream_t s);
 
-// MXFP4 weights with few routed rows per expert (skinny_fp4.cu): the codes
-// are decoded in registers; no expansion pass.
-bool skinny_fp4_applies(const moe_dims_t& d);
-moe_status_t launch_mlp1_fp4_skinny(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
+// MXFP4 weights with few routed rows per expert (stream_fp4.cu): the codes
+// are streamed from HBM once and decoded on chip into tcgen05 operands; no
+// expansion pass. Applies when the experts average at most 16 routed rows.
+bool stream_fp4_applies(const moe_dims_t& d);
+moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
                                     const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
                                     uint16_t* tok16, int* status, cudaStream_t s);
-moe_status_t launch_mlp2_fp4_skinny(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
+moe_status_t launch_mlp2_fp4_stream(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
                                     const int32_t* offsets, const float* topk_w, const uint8_t* codes,
                                     const uint8_t* scales, const uint16_t* b2, float* o_perm, uint16_t* tok16,
                                     int* status, cudaStream_t s);

@@ -48,3 +48,23 @@ def test_single_rank_is_identity():
     assert bench.max_over_ranks([1.0, 2.0], 1) == [1.0, 2.0]
     ms, value = bench.step_throughput(1000.0, 10, 8192, 1)
     assert ms == 100.0 and value == pytest.approx(81920.0)
+
+
+def test_profile_traffic_is_read_for_the_profiled_kernel_sources(tmp_path, monkeypatch):
+    # the committed ncu summary carries the hash of the GEMM sources it was
+    # taken on; the bench reports its DRAM bytes only while that hash matches
+    p = os.path.join(bench.ROOT, "profiles", "mlp1_gptoss20b_ncu.md")
+    text = open(p).read()
+    fake = tmp_path / "profiles"
+    fake.mkdir()
+    (fake / "mlp1_gptoss20b_ncu.md").write_text(text)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    import re
+
+    sha = re.search(r"kernel_sources_sha256_16: `([0-9a-f]{16})`", text).group(1)
+    nbytes = int(re.search(r"dram_bytes_per_launch: `(\d+)`", text).group(1))
+    monkeypatch.setattr(bench, "gemm_source_hash", lambda: sha)
+    assert bench.traffic_from_profile() == nbytes
+    # a summary taken on other kernel sources is ignored
+    monkeypatch.setattr(bench, "gemm_source_hash", lambda: "f" * 16)
+    assert bench.traffic_from_profile() is None

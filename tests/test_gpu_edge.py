@@ -10,14 +10,14 @@ import torch
 import mixture_experts_ffn_layer_b200 as moe
 import oracle
 import synthetic
-from helpers import TOL_BF16, assert_close_rms, run_stages
+from helpers import TOL_BF16, TOL_MXFP4, assert_close_rms, run_stages
 
 pytestmark = pytest.mark.gpu
 
 BF16 = torch.bfloat16
 
 
-def _check_full(inp):
+def _check_full(inp, tol=TOL_BF16):
     run = run_stages(inp)
     assert run.status == 0, moe.status_str(run.status)
     s = inp.shape
@@ -27,8 +27,9 @@ def _check_full(inp):
     counts, offsets, perm, inv = oracle.permute(idx_ref, s.E)
     for a, b in ((run.counts, counts), (run.offsets, offsets), (run.perm, perm), (run.inv, inv)):
         assert torch.equal(a.cpu(), b)
-    _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, return_exact=True)
-    assert_close_rms(run.y, y_ref, TOL_BF16)
+    _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, return_exact=True,
+                                 W1_scales=inp.W1_scales, W2_scales=inp.W2_scales)
+    assert_close_rms(run.y, y_ref, tol)
     return run
 
 
@@ -44,6 +45,35 @@ def _check_full(inp):
 def test_shapes(T, D, E, k, I):
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", reject=oracle.gap_reject())
     _check_full(inp)
+
+
+@pytest.mark.parametrize("T,D,E,k,I", [
+    (8, 64, 4, 2, 64),      # one 64-element K step, a partial 128-row weight block
+    (40, 192, 8, 2, 320),   # three K steps, 2.5 weight blocks per expert
+    (1, 128, 32, 4, 64),    # one token
+    (96, 256, 24, 1, 192),  # non-power-of-two E
+])
+def test_mxfp4_weight_streaming_shapes(T, D, E, k, I):
+    # at most 16 routed rows per expert on average: the MXFP4 weight-streaming kernels
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + 7 * E, device="cuda", wfmt="mxfp4",
+                                reject=oracle.gap_reject())
+    _check_full(inp, TOL_MXFP4)
+
+
+def test_mxfp4_hot_expert_several_passes():
+    # one expert takes most tokens: its rows span several 32-row passes, the
+    # last one ragged, while the other experts keep a few rows
+    T, D, E, k, I = 120, 128, 16, 2, 128
+    base = synthetic.make_custom(T, D, E, k, I, seed=11, wfmt="mxfp4")
+    br = torch.zeros(E)
+    br[5] = 6.0
+    br = br.to(BF16)
+    keep = ~oracle.gap_reject()(base.x, base.Wr, br, k)
+    x = base.x[keep].contiguous()
+    shape = synthetic.LayerShape("custom", x.shape[0], D, E, k, I, wfmt="mxfp4")
+    inp = dataclasses.replace(base, shape=shape, x=x, br=br).to("cuda")
+    run = _check_full(inp, TOL_MXFP4)
+    assert int(run.counts.max()) > 64
 
 
 def test_empty_experts():
