@@ -11,7 +11,7 @@ namespace {
 
 struct WsLayout {
   size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, w1_deq, w2_deq, tok16,
-      total;
+      route_partial, total;
 };
 
 WsLayout ws_layout(const moe_dims_t& d) {
@@ -33,6 +33,8 @@ WsLayout ws_layout(const moe_dims_t& d) {
   L.x_perm = take(static_cast<size_t>(R) * d.D * 2);
   L.h = take(static_cast<size_t>(R) * d.I * 2);
   L.o_perm = take(static_cast<size_t>(R) * d.D * 4);
+  if (route_splits(d) > 1)  // K-split router: fp32 partial logits per split
+    L.route_partial = take(static_cast<size_t>(route_splits(d)) * d.T * ((d.E + 15) / 16 * 16) * 4);
   if (stream_fp4_applies(d)) {
     // routed rows (x_perm, then h) in f16 for the weight-streaming MXFP4 kernels
     L.tok16 = take(static_cast<size_t>(R) * (d.D > d.I ? d.D : d.I) * 2);
@@ -127,8 +129,10 @@ moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, cons
   MOE_REQUIRE(x && Wr && br && topk_idx && topk_w);
   MOE_REQUIRE(aligned32(x) && aligned32(Wr));
   MOE_TRY(check_ws(d, ws, ws_bytes));
+  const WsLayout L = ws_layout(d);
+  float* partial = route_splits(d) > 1 ? at<float>(ws, L.route_partial) : nullptr;
   return cuda_status(
-      launch_route(d, x, Wr, br, topk_idx, topk_w, status_word(ws), static_cast<cudaStream_t>(stream)));
+      launch_route(d, x, Wr, br, topk_idx, topk_w, partial, status_word(ws), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets, int32_t* perm,

@@ -47,8 +47,12 @@ constexpr int kPermThreads = 256;
 inline int perm_blocks(int64_t R, int chunk = kPermChunk) { return static_cast<int>((R + chunk - 1) / chunk); }
 
 // Kernel launchers (defined in the .cu files).
+// Router (route.cu). With route_splits(d) > 1 the contraction is split along
+// K and `partial` holds route_splits(d) * T * n_pad fp32 (n_pad = E rounded
+// up to 16).
+int route_splits(const moe_dims_t& d);
 cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
-                         int32_t* topk_idx, float* topk_w, int* status, cudaStream_t s);
+                         int32_t* topk_idx, float* topk_w, float* partial, int* status, cudaStream_t s);
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
                            int chunk = kPermChunk);

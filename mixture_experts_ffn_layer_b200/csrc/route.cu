@@ -12,6 +12,11 @@
 // it streams the token's E logits out of TMEM, adds the bias, keeps a sorted
 // top-k in registers and writes the normalised gate weights. x is read once
 // from HBM; Wr stays L2-resident.
+// With fewer 128-token tiles than SMs (decode batches) the contraction is also
+// split along K across CTAs so that the SMs all stream x: each split writes
+// its fp32 partial logits, and a second kernel (one warp per token) sums the
+// splits in a fixed order, adds the bias and takes the same top-k / softmax,
+// so the result is deterministic for given sizes.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -32,6 +37,9 @@ struct RouteParams {
   int n_pad;        // MMA N: E rounded up to a multiple of 16
   int stages;       // TMA ring depth (as many as fit: few CTAs stream all of x)
   uint32_t tmem_cols;
+  int kb_per;       // K blocks per split (all of them when there is one split)
+  int ksplit;       // number of K splits (gridDim.y)
+  float* partial;   // (ksplit, T, n_pad) fp32 partial logits when ksplit > 1
   const uint16_t* br;
   int32_t* topk_idx;
   float* topk_w;
@@ -58,6 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t done_bar = bar0 + 8u * (2 * kMaxStages + 1);
   const int t0 = blockIdx.x * BM;
   const int KB = (p.D + BK - 1) / BK;
+  const int kb0 = blockIdx.y * p.kb_per, kb1 = min(KB, kb0 + p.kb_per);
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -86,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool failed = false;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, kWaitNs)) {
           failed = true;
           break;
@@ -123,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool failed = false;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, kWaitNs)) {
           failed = true;
           break;
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
           mma_bf16(tmem_base, desc_kmajor_sw128(a_addr + kk * 32), desc_kmajor_sw128(b_addr + kk * 32), idesc,
-                   (kb | kk) != 0 ? 1u : 0u);
+                   (kb != kb0 || kk != 0) ? 1u : 0u);
         tc_commit(empty_bar(stage));
         if (++stage == kStages) {
           stage = 0;
@@ -155,7 +164,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int t = t0 + q * 32 + lane;
     const bool ok = mbar_wait_bounded(tfull_bar, 0, abort_flag, kWaitNs);
-    if (__all_sync(0xffffffffu, ok)) {
+    if (__all_sync(0xffffffffu, ok) && p.ksplit > 1) {
+      // partial logits of this K split: the token's n_pad accumulator columns
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      float* dst = p.partial + (static_cast<int64_t>(blockIdx.y) * p.T + t) * p.n_pad;
+      for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (c0 + 8 * j < p.n_pad) tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+        tmem_ld_wait();
+        if (t < p.T) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c0 + 4 * j < p.n_pad)
+              *reinterpret_cast<uint4*>(dst + c0 + 4 * j) = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+    } else if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       float topv[kMaxK];
       int tope[kMaxK];
@@ -226,10 +253,104 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Sum of the K splits' partial logits (split order 0, 1, ...), bias, top-k
+// and softmax over the chosen logits; one warp per token, lanes over experts.
+// Ties go to the lower expert index, as in the fused epilogue.
+__global__ void __launch_bounds__(128) route_reduce_topk_kernel(const RouteParams p) {
+  const int t = blockIdx.x * 4 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (t >= p.T) return;
+  constexpr int kPerLane = 8;  // E <= 256
+  float v[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = -FLT_MAX;
+    if (e < p.E) {
+      // fixed order sp = 0, 1, ...; loads issued eight at a time
+      const float* src = p.partial + static_cast<int64_t>(t) * p.n_pad + e;
+      const int64_t stride = static_cast<int64_t>(p.T) * p.n_pad;
+      float acc = 0.f;
+      int sp = 0;
+      for (; sp + 8 <= p.ksplit; sp += 8) {
+        float part[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[u] = src[(sp + u) * stride];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc += part[u];
+      }
+      for (; sp < p.ksplit; ++sp) acc += src[sp * stride];
+      v[i] = acc + bf16_bits_to_float(__ldg(p.br + e));
+    }
+  }
+  uint32_t taken = 0;
+  float topv[kMaxK];
+  int tope[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    topv[j] = -FLT_MAX;
+    tope[j] = 0x7fffffff;
+    if (j >= p.k) continue;
+    // this lane's best untaken candidate, then the warp's (value desc, index asc)
+    float bv = -FLT_MAX;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const int e = lane + 32 * i;
+      if (e < p.E && !(taken >> i & 1u) && v[i] > bv) {  // strict: lower index wins ties
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    topv[j] = bv;
+    tope[j] = be;
+    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
+  }
+  if (lane == 0) {
+    float ex[kMaxK], denom = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      ex[j] = j < p.k ? __expf(topv[j] - topv[0]) : 0.f;
+      denom += ex[j];
+    }
+    const float inv = 1.0f / denom;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < p.k) {
+        p.topk_idx[static_cast<int64_t>(t) * p.k + j] = tope[j];
+        p.topk_w[static_cast<int64_t>(t) * p.k + j] = ex[j] * inv;
+      }
+    }
+  }
+}
+
 }  // namespace
 
+int route_splits(const moe_dims_t& d) {
+  // With few token tiles, enough K splits that tiles x splits cover the SMs
+  // (one wave of 148 on B200); fixed by the sizes, so results do not depend on
+  // the device. Measured on B200: at 64 tiles (8192 tokens) two splits cost
+  // more (partials + second launch) than they save, at 1 tile (64 tokens)
+  // 45 splits save ~5 us; so only batches of at most 18 tiles split.
+  const int tiles = (d.T + BM - 1) / BM, KB = (d.D + BK - 1) / BK;
+  if (tiles * 8 > 148) return 1;
+  int sp = 148 / tiles;
+  if (sp > KB) sp = KB;
+  if (sp < 1) sp = 1;
+  const int per = (KB + sp - 1) / sp;
+  return (KB + per - 1) / per;
+}
+
 cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
-                         int32_t* topk_idx, float* topk_w, int* status, cudaStream_t s) {
+                         int32_t* topk_idx, float* topk_w, float* partial, int* status, cudaStream_t s) {
   RouteParams p{};
   p.T = d.T;
   p.D = d.D;
@@ -243,17 +364,24 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
   p.topk_idx = topk_idx;
   p.topk_w = topk_w;
   p.status = status;
+  const int KB = (d.D + BK - 1) / BK;
+  p.ksplit = route_splits(d);
+  p.kb_per = (KB + p.ksplit - 1) / p.ksplit;
+  p.partial = partial;
+  if (p.ksplit > 1 && !partial) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap_bf16(&tx, x, d.D, d.T, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tw, Wr, d.D, d.E, p.n_pad)) return cudaErrorInvalidValue;
   const size_t stage_bytes = kABytes + static_cast<size_t>(p.n_pad) * BK * 2;
   p.stages = static_cast<int>((200 * 1024) / stage_bytes);
   if (p.stages > kMaxStages) p.stages = kMaxStages;
+  if (p.stages > p.kb_per) p.stages = p.kb_per < 2 ? 2 : p.kb_per;
   const size_t smem = 1024 + p.stages * stage_bytes + 8 * (2 * kMaxStages + 2) + 16;
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  route_tc_kernel<<<(d.T + BM - 1) / BM, kThreads, smem, s>>>(tx, tw, p);
+  route_tc_kernel<<<dim3((d.T + BM - 1) / BM, p.ksplit), kThreads, smem, s>>>(tx, tw, p);
+  if (p.ksplit > 1) route_reduce_topk_kernel<<<(d.T + 3) / 4, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -92,8 +92,9 @@ def test_empty_experts():
     assert int((run.counts == 0).sum()) >= 10
 
 
-def test_exact_ties_pick_lower_index():
-    T, D, E, k, I = 96, 64, 6, 3, 64
+@pytest.mark.parametrize("D", [64, 256])  # 256: the router's K-split path (partial logits + reduce)
+def test_exact_ties_pick_lower_index(D):
+    T, E, k, I = 96, 6, 3, 64
     g = torch.Generator().manual_seed(5)
     x = torch.randint(-2, 3, (T, D), generator=g).to(BF16)
     base = torch.randint(-1, 2, (3, D), generator=g)
