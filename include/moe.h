@@ -68,8 +68,20 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1 } moe_wfmt_t;
 
 /* T tokens, D model dim, E experts, top-k, I expert intermediate dim, and the
  * expert-weight format (moe_wfmt_t). R = T*k routed rows. */
+/* Activation between mlp1 and mlp2, on the gate half g and up half u of mlp1's
+ * output (rows [0,I) and [I,2I) of W1):
+ *   MOE_ACT_SWIGLU:  h = silu(g) * u, silu(g) = g / (1 + e^-g)
+ *   MOE_ACT_GPTOSS:  the GPT-OSS variant (torchtitan GPT-OSS guide, paragraph
+ *     on the grouped experts' SwiGLU variant): gc = min(g, act_limit),
+ *     uc = min(max(u, -act_limit), act_limit), h = gc * sigmoid(act_alpha * gc) * (uc + 1).
+ *     The pages do not give alpha and limit; the caller does (act_limit may be
+ *     +inf for no clamping). Ignored for MOE_ACT_SWIGLU. */
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GPTOSS = 1 } moe_act_t;
+
 typedef struct {
   int32_t T, D, E, k, I, wfmt;
+  int32_t act;                /* moe_act_t */
+  float act_alpha, act_limit; /* MOE_ACT_GPTOSS only */
 } moe_dims_t;
 
 /* An expert weight tensor of logical shape (E, N, K), K the reduction dim.
@@ -117,7 +129,8 @@ MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* 
 
 /* Grouped mlp1 + bias + SwiGLU over the expert segments of x_perm:
  * for r in [offsets[e], offsets[e+1]):
- *   u = W1[e] . x_perm[r] + b1[e] (fp32 accumulate), h[r,i] = bf16(silu(u[i]) * u[I+i]).
+ *   u = W1[e] . x_perm[r] + b1[e] (fp32 accumulate), h[r,i] = bf16(act(u[i], u[I+i]))
+ *   with act = d.act (plain SwiGLU or the GPT-OSS variant, see moe_act_t).
  *   x_perm (R,D) bf16, offsets (E+1), W1 (E,2I,D), b1 (E,2I) bf16 -> h (R,I) bf16.
  * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile).
  * MXFP4 weights: with T*k <= 16*E (a few rows per expert) the codes are

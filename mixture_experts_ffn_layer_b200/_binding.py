@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 MOE_W_BF16, MOE_W_MXFP4 = 0, 1
+MOE_ACT_SWIGLU, MOE_ACT_GPTOSS = 0, 1
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA",
     5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_DEVICE_BOUNDS",
@@ -34,7 +35,8 @@ class MoeError(RuntimeError):
 
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("D", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("I", ctypes.c_int32), ("wfmt", ctypes.c_int32)]
+                ("I", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("act_alpha", ctypes.c_float), ("act_limit", ctypes.c_float)]
 
 
 class Weight(ctypes.Structure):
@@ -81,8 +83,8 @@ def load(path: str = LIB_PATH):
     return L
 
 
-def dims(T, D, E, k, I, wfmt=MOE_W_BF16) -> Dims:
-    return Dims(T, D, E, k, I, wfmt)
+def dims(T, D, E, k, I, wfmt=MOE_W_BF16, act=MOE_ACT_SWIGLU, act_alpha=1.0, act_limit=float("inf")) -> Dims:
+    return Dims(T, D, E, k, I, wfmt, act, act_alpha, act_limit)
 
 
 def _p(t: Optional[torch.Tensor]):

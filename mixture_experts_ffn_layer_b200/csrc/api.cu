@@ -2,6 +2,8 @@
 // enqueueing of the kernels of route.cu, permute.cu, grouped_gemm.cu and
 // mxfp4.cu on the caller's stream. No host synchronisation except in
 // moe_read_device_status.
+#include <cmath>
+
 #include "common.cuh"
 
 #include <stdint.h>
@@ -112,6 +114,9 @@ moe_status_t moe_check_dims(moe_dims_t d) {
   if (d.T <= 0 || d.D <= 0 || d.E <= 0 || d.k <= 0 || d.I <= 0) return MOE_ERR_INVALID_ARG;
   if (d.k > d.E) return MOE_ERR_INVALID_ARG;
   if (d.wfmt != MOE_W_BF16 && d.wfmt != MOE_W_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (d.act != MOE_ACT_SWIGLU && d.act != MOE_ACT_GPTOSS) return MOE_ERR_INVALID_ARG;
+  // GPT-OSS variant: a finite alpha and a limit > 0 (+inf allowed: no clamping)
+  if (d.act == MOE_ACT_GPTOSS && (!std::isfinite(d.act_alpha) || !(d.act_limit > 0.0f))) return MOE_ERR_INVALID_ARG;
   if (d.E > 256 || d.k > 8) return MOE_ERR_UNSUPPORTED;
   if (d.D % 64 || d.I % 64 || d.D > 16384 || d.I > 16384) return MOE_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d.T) * d.k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;

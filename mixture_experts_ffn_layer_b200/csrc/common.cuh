@@ -46,6 +46,24 @@ constexpr int kPermThreads = 256;
 
 inline int perm_blocks(int64_t R, int chunk = kPermChunk) { return static_cast<int>((R + chunk - 1) / chunk); }
 
+// The activation between mlp1 and mlp2 on gate g and up u (moe_act_t in
+// moe.h): plain SwiGLU silu(g) * u, or the GPT-OSS variant with the gate
+// clamped from above at `limit`, sigmoid(alpha * gate), up clipped to
+// [-limit, limit] plus 1.
+struct Act {
+  int kind;
+  float alpha, limit;
+};
+
+__device__ __forceinline__ float glu_act(float g, float u, const Act& a) {
+  if (a.kind == MOE_ACT_SWIGLU) return __fdividef(g, 1.0f + __expf(-g)) * u;
+  const float gc = fminf(g, a.limit);
+  const float uc = fminf(fmaxf(u, -a.limit), a.limit);
+  return __fdividef(gc, 1.0f + __expf(-a.alpha * gc)) * (uc + 1.0f);
+}
+
+inline Act act_of(const moe_dims_t& d) { return Act{d.act, d.act_alpha, d.act_limit}; }
+
 // Kernel launchers (defined in the .cu files).
 // Router (route.cu). With route_splits(d) > 1 the contraction is split along
 // K and `partial` holds route_splits(d) * T * n_pad fp32 (n_pad = E rounded

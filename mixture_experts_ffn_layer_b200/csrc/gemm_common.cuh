@@ -22,6 +22,7 @@ struct GemmParams {
   const float* topk_w;
   void* out;  // h (R, I) bf16 for mlp1; o_perm (R, D) fp32 for mlp2
   int* status;
+  Act act;    // mlp1's activation
 };
 
 // Tile `tile` -> (expert e, column tile nt, row tile mt) for row tiles of bm
@@ -53,6 +54,7 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 }
 
 // Fused epilogue of one accumulator tile for the thread's row: bias + SwiGLU
+// (or its GPT-OSS variant)
 // into h (bf16), or bias times the gate weight into o (fp32). tbase is the
 // TMEM address of the thread's lane at column 0 of the accumulator; row is
 // the routed row, valid = row inside the expert segment.
@@ -88,7 +90,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
           for (int i = 0; i < 8; ++i) {
             const float gate = __uint_as_float(g[8 * j + i]) + gb[i];
             const float up = __uint_as_float(u[8 * j + i]) + ub[i];
-            hv[i] = __fdividef(gate, 1.0f + __expf(-gate)) * up;
+            hv[i] = glu_act(gate, up, p.act);
           }
           if (valid) {
             uint4 v;

@@ -314,6 +314,7 @@ moe_status_t launch_mlp1(const moe_dims_t& d, const uint16_t* x_perm, const int3
   p.R = R;
   p.offsets = offsets;
   p.bias = b1;
+  p.act = act_of(d);
   p.out = h;
   p.status = status;
   return launch_gemm<true>(ta, tb, p, s);

@@ -331,6 +331,7 @@ moe_status_t launch_mlp1_pair(const moe_dims_t& d, const uint16_t* x_perm, const
   p.R = R;
   p.offsets = offsets;
   p.bias = b1;
+  p.act = act_of(d);
   p.out = h;
   p.status = status;
   pp.n_half = nh;

@@ -77,6 +77,7 @@ struct StreamParams {
   const float* topk_w;
   void* out;              // h (R, I) bf16 or o_perm (R, D) fp32
   int* status;
+  Act act;     // mlp1's activation
   int stages;  // pipeline depth that fits shared memory next to the block scales
 };
 
@@ -402,8 +403,7 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
           const float g = __uint_as_float(vg[i]) * fg + bg;
           if (kSwiGLU) {
             const float u = __uint_as_float(vu[i]) * fu + bu;
-            static_cast<uint16_t*>(p.out)[row * p.n_out + col] =
-                float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * u);
+            static_cast<uint16_t*>(p.out)[row * p.n_out + col] = float_to_bf16_bits(glu_act(g, u, p.act));
           } else {
             const int32_t a = p.perm[row];
             float wgt = 0.f;
@@ -511,6 +511,7 @@ moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm,
   p.scales = scales;
   p.bias = b1;
   p.in_scale = 1.0f;
+  p.act = act_of(d);
   p.out = h;
   p.status = status;
   CUtensorMap tm;

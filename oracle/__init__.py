@@ -49,10 +49,11 @@ def lib():
         L.oracle_dequant_mxfp4.argtypes = [c_vp, c_vp, c_i64, c_i64, c_vp]
         L.oracle_route.argtypes = [c_i64, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
         L.oracle_permute.argtypes = [c_i64, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]
-        L.oracle_ffn_tokens.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp,
-                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp]
-        L.oracle_forward.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp,
-                                     c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
+        c_dbl = ctypes.c_double
+        L.oracle_ffn_tokens.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_int, c_dbl, c_dbl, c_vp, c_vp,
+                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp]
+        L.oracle_forward.argtypes = [c_i64, c_int, c_int, c_int, c_int, c_int, c_int, c_dbl, c_dbl, c_vp, c_vp,
+                                     c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
         for f in ("oracle_dequant_mxfp4", "oracle_route", "oracle_permute", "oracle_ffn_tokens", "oracle_forward"):
             getattr(L, f).restype = c_int
         _lib = L
@@ -120,11 +121,17 @@ def permute(topk_idx, E: int):
     return counts, offsets, perm, inv
 
 
+ACT_SWIGLU, ACT_GPTOSS = 0, 1
+
+
 def ffn_tokens(x, topk_idx, topk_w, W1, b1, W2, b2, tokens: Optional[Sequence[int]] = None,
-               W1_scales=None, W2_scales=None, return_o: bool = False, return_exact: bool = False):
+               W1_scales=None, W2_scales=None, return_o: bool = False, return_exact: bool = False,
+               act=(ACT_SWIGLU, 1.0, float("inf"))):
     """Expert FFN + weighted combine for ``tokens`` (default all) -> y (n, D) bf16
     [and o (n, k, D) float64, the unweighted expert outputs]
-    [and y_exact (n, D) float64, y before its final bf16 rounding]."""
+    [and y_exact (n, D) float64, y before its final bf16 rounding].
+    ``act`` = (kind, alpha, limit): plain SwiGLU (kind 0) or the GPT-OSS
+    variant (kind 1, clamp at ``limit``, sigmoid(alpha * gate), up + 1)."""
     x, idx, w = _cpu(x), _cpu(topk_idx).to(torch.int32), _cpu(topk_w).float()
     W1, b1, W2, b2 = _cpu(W1), _cpu(b1), _cpu(W2), _cpu(b2)
     W1s, W2s = _cpu(W1_scales), _cpu(W2_scales)
@@ -141,8 +148,9 @@ def ffn_tokens(x, topk_idx, topk_w, W1, b1, W2, b2, tokens: Optional[Sequence[in
     y = torch.empty((n, D), dtype=torch.int16)
     o = torch.empty((n, k, D), dtype=torch.float64) if return_o else None
     ye = torch.empty((n, D), dtype=torch.float64) if return_exact else None
-    _check(lib().oracle_ffn_tokens(T, D, E, k, I, wfmt, _ptr(x), _ptr(idx), _ptr(w), _ptr(W1), _ptr(W1s), _ptr(b1),
-                                   _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(tok), n, _ptr(y), _ptr(o), _ptr(ye)),
+    _check(lib().oracle_ffn_tokens(T, D, E, k, I, wfmt, int(act[0]), float(act[1]), float(act[2]), _ptr(x), _ptr(idx),
+                                   _ptr(w), _ptr(W1), _ptr(W1s), _ptr(b1), _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(tok), n,
+                                   _ptr(y), _ptr(o), _ptr(ye)),
            "ffn_tokens")
     out = [y.view(torch.bfloat16)]
     if return_o:
@@ -152,7 +160,7 @@ def ffn_tokens(x, topk_idx, topk_w, W1, b1, W2, b2, tokens: Optional[Sequence[in
     return tuple(out) if len(out) > 1 else out[0]
 
 
-def forward(x, Wr, br, W1, b1, W2, b2, k: int, W1_scales=None, W2_scales=None):
+def forward(x, Wr, br, W1, b1, W2, b2, k: int, W1_scales=None, W2_scales=None, act=(ACT_SWIGLU, 1.0, float("inf"))):
     """The whole layer -> (y (T,D) bf16, topk_idx (T,k) int32, topk_w (T,k) float32)."""
     x, Wr, br = _cpu(x), _cpu(Wr), _cpu(br)
     W1, b1, W2, b2 = _cpu(W1), _cpu(b1), _cpu(W2), _cpu(b2)
@@ -164,8 +172,9 @@ def forward(x, Wr, br, W1, b1, W2, b2, k: int, W1_scales=None, W2_scales=None):
     y = torch.empty((T, D), dtype=torch.int16)
     idx = torch.empty((T, k), dtype=torch.int32)
     w = torch.empty((T, k), dtype=torch.float32)
-    _check(lib().oracle_forward(T, D, E, k, I, wfmt, _ptr(x), _ptr(Wr), _ptr(br), _ptr(W1), _ptr(W1s), _ptr(b1),
-                                _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(y), _ptr(idx), _ptr(w)), "forward")
+    _check(lib().oracle_forward(T, D, E, k, I, wfmt, int(act[0]), float(act[1]), float(act[2]), _ptr(x), _ptr(Wr),
+                                _ptr(br), _ptr(W1), _ptr(W1s), _ptr(b1), _ptr(W2), _ptr(W2s), _ptr(b2), _ptr(y), _ptr(idx),
+                                _ptr(w)), "forward")
     return y.view(torch.bfloat16), idx, w
 
 

@@ -19,7 +19,15 @@
 //      "grouped matrix multiplication": weights stored (num_experts, out_dim,
 //      in_dim), mlp1 then SwiGLU then mlp2, each with a bias):
 //        u[n] = sum_d x[t,d] * W1[e,n,d] + b1[e,n],   n < 2I
-//        h[i] = bf16( silu(u[i]) * u[I+i] ),          i < I, silu(g) = g/(1+e^-g)
+//        h[i] = bf16( act(u[i], u[I+i]) ),            i < I
+//      act = plain SwiGLU silu(g) * u with silu(g) = g/(1+e^-g) (act 0), or
+//      the GPT-OSS variant (act 1; torchtitan GPT-OSS guide, paragraph on
+//      GptOssGroupedExperts' SwiGLU variant): the gate branch is clamped from
+//      above at `limit` and multiplied by sigmoid(alpha * gate), the linear
+//      branch is clipped to [-limit, limit] and offset by 1:
+//        gc = min(g, limit), uc = min(max(u, -limit), limit),
+//        act = gc * sigmoid(alpha * gc) * (uc + 1);
+//      alpha and limit are the caller's (the pages do not give them).
 //        o[c] = sum_i h[i] * W2[e,c,i] + b2[e,c],     c < D
 //      rows [0,I) of W1[e] are the gate half, rows [I,2I) the up half.
 //   5. weighted combine (from-scratch GPT-OSS write-up, "model flow" diagram,
@@ -110,6 +118,17 @@ struct Weights {
 
 double silu(double g) { return g / (1.0 + std::exp(-g)); }
 
+struct Act {
+  int kind;  // 0 plain SwiGLU, 1 GPT-OSS variant
+  double alpha, limit;
+  double operator()(double g, double u) const {
+    if (kind == 0) return silu(g) * u;
+    const double gc = std::min(g, limit);
+    const double uc = std::min(std::max(u, -limit), limit);
+    return gc / (1.0 + std::exp(-alpha * gc)) * (uc + 1.0);
+  }
+};
+
 void route_token(int64_t t, int D, int E, int k, const uint16_t* x, const uint16_t* Wr,
                  const uint16_t* br, float* logits_row, int32_t* idx_row, float* w_row) {
   std::vector<float> l(E);
@@ -138,7 +157,7 @@ void route_token(int64_t t, int D, int E, int k, const uint16_t* x, const uint16
 
 // Expert FFN output o (length D, double) of token row x_row for expert e.
 void expert_ffn(const uint16_t* x_row, int D, int I, int64_t e, const Weights& W1, const uint16_t* b1,
-                const Weights& W2, const uint16_t* b2, std::vector<double>& u, std::vector<double>& h,
+                const Weights& W2, const uint16_t* b2, const Act& act, std::vector<double>& u, std::vector<double>& h,
                 std::vector<double>& o) {
   const int64_t twoI = 2 * static_cast<int64_t>(I);
   for (int64_t n = 0; n < twoI; ++n) {
@@ -146,7 +165,7 @@ void expert_ffn(const uint16_t* x_row, int D, int I, int64_t e, const Weights& W
     for (int d = 0; d < D; ++d) acc += bf16_to_double(x_row[d]) * W1.at(e, n, d);
     u[n] = acc + bf16_to_double(b1[e * twoI + n]);
   }
-  for (int i = 0; i < I; ++i) h[i] = bf16_to_double(double_to_bf16(silu(u[i]) * u[I + i]));
+  for (int i = 0; i < I; ++i) h[i] = bf16_to_double(double_to_bf16(act(u[i], u[I + i])));
   for (int c = 0; c < D; ++c) {
     double acc = 0.0;
     for (int i = 0; i < I; ++i) acc += h[i] * W2.at(e, c, i);
@@ -221,11 +240,14 @@ int oracle_permute(int64_t T, int E, int k, const int32_t* topk_idx, int32_t* co
 // y_out: ntok x D bf16. o_out (nullable): ntok x k x D doubles, the unweighted
 // expert outputs o_j. y_exact (nullable): ntok x D doubles, the weighted sum
 // before its final bf16 rounding.
-int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, const uint16_t* x,
-                      const int32_t* topk_idx, const float* topk_w, const void* W1, const uint8_t* W1_scales,
-                      const uint16_t* b1, const void* W2, const uint8_t* W2_scales, const uint16_t* b2,
-                      const int64_t* tokens, int64_t ntok, uint16_t* y_out, double* o_out, double* y_exact) {
+int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, int act_kind, double act_alpha,
+                      double act_limit, const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                      const void* W1, const uint8_t* W1_scales, const uint16_t* b1, const void* W2,
+                      const uint8_t* W2_scales, const uint16_t* b2, const int64_t* tokens, int64_t ntok,
+                      uint16_t* y_out, double* o_out, double* y_exact) {
   if (!dims_ok(T, D, E, k, I)) return 1;
+  if (act_kind != 0 && act_kind != 1) return 1;
+  const Act act{act_kind, act_alpha, act_limit};
   if (wfmt != 0 && wfmt != 1) return 1;
   if (wfmt == 1 && (D % 32 || I % 32)) return 1;
   Weights w1{wfmt, static_cast<const uint16_t*>(W1), static_cast<const uint8_t*>(W1), W1_scales, 2 * static_cast<int64_t>(I), D};
@@ -250,7 +272,7 @@ int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, const uin
           err = 2;
           break;
         }
-        expert_ffn(x + t * D, D, I, e, w1, b1, w2, b2, u, h, o);
+        expert_ffn(x + t * D, D, I, e, w1, b1, w2, b2, act, u, h, o);
         double wj = static_cast<double>(topk_w[t * k + j]);
         for (int c = 0; c < D; ++c) y[c] += wj * o[c];
         if (o_out)
@@ -265,16 +287,16 @@ int oracle_ffn_tokens(int64_t T, int D, int E, int k, int I, int wfmt, const uin
 }
 
 // The whole layer for all tokens: route, then FFN + combine.
-int oracle_forward(int64_t T, int D, int E, int k, int I, int wfmt, const uint16_t* x, const uint16_t* Wr,
-                   const uint16_t* br, const void* W1, const uint8_t* W1_scales, const uint16_t* b1,
-                   const void* W2, const uint8_t* W2_scales, const uint16_t* b2, uint16_t* y,
-                   int32_t* topk_idx, float* topk_w) {
+int oracle_forward(int64_t T, int D, int E, int k, int I, int wfmt, int act_kind, double act_alpha,
+                   double act_limit, const uint16_t* x, const uint16_t* Wr, const uint16_t* br, const void* W1,
+                   const uint8_t* W1_scales, const uint16_t* b1, const void* W2, const uint8_t* W2_scales,
+                   const uint16_t* b2, uint16_t* y, int32_t* topk_idx, float* topk_w) {
   int rc = oracle_route(T, D, E, k, x, Wr, br, nullptr, topk_idx, topk_w);
   if (rc) return rc;
   std::vector<int64_t> tokens(T);
   for (int64_t t = 0; t < T; ++t) tokens[t] = t;
-  return oracle_ffn_tokens(T, D, E, k, I, wfmt, x, topk_idx, topk_w, W1, W1_scales, b1, W2, W2_scales, b2,
-                           tokens.data(), T, y, nullptr, nullptr);
+  return oracle_ffn_tokens(T, D, E, k, I, wfmt, act_kind, act_alpha, act_limit, x, topk_idx, topk_w, W1, W1_scales,
+                           b1, W2, W2_scales, b2, tokens.data(), T, y, nullptr, nullptr);
 }
 
 }  // extern "C"

@@ -30,16 +30,19 @@ class GpuRun:
     status: int
 
 
-def dims_of(inp: synthetic.LayerInputs):
+SWIGLU = (moe.MOE_ACT_SWIGLU, 1.0, float("inf"))  # (act, alpha, limit); oracle.ACT_* use the same codes
+
+
+def dims_of(inp: synthetic.LayerInputs, act=SWIGLU):
     s = inp.shape
-    return moe.dims(s.T, s.D, s.E, s.k, s.I, moe.MOE_W_MXFP4 if s.wfmt == "mxfp4" else moe.MOE_W_BF16)
+    return moe.dims(s.T, s.D, s.E, s.k, s.I, moe.MOE_W_MXFP4 if s.wfmt == "mxfp4" else moe.MOE_W_BF16, *act)
 
 
-def run_stages(inp: synthetic.LayerInputs) -> GpuRun:
+def run_stages(inp: synthetic.LayerInputs, act=SWIGLU) -> GpuRun:
     """Every stage through its own C-ABI entry point, intermediates kept."""
     s = inp.shape
     dev = inp.x.device
-    d = dims_of(inp)
+    d = dims_of(inp, act)
     ws = moe.alloc_workspace(d, device=dev)
     R = s.T * s.k
     i32 = dict(dtype=torch.int32, device=dev)
@@ -63,9 +66,9 @@ def run_stages(inp: synthetic.LayerInputs) -> GpuRun:
     return GpuRun(topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, y, status)
 
 
-def run_forward(inp: synthetic.LayerInputs) -> torch.Tensor:
+def run_forward(inp: synthetic.LayerInputs, act=SWIGLU) -> torch.Tensor:
     s = inp.shape
-    d = dims_of(inp)
+    d = dims_of(inp, act)
     ws = moe.alloc_workspace(d, device=inp.x.device)
     y = torch.empty((s.T, s.D), dtype=torch.bfloat16, device=inp.x.device)
     moe.moe_forward(d, inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws, W1_scales=inp.W1_scales,

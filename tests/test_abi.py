@@ -41,6 +41,14 @@ def test_check_dims_supported_set():
     assert moe.check_dims(moe.dims(8, 64, 16, 9, 64)) == 2  # k > 8
     assert moe.check_dims(moe.dims(8, 96, 4, 2, 64)) == 2  # D % 64
     assert moe.check_dims(moe.dims(8, 64, 4, 2, 100)) == 2  # I % 64
+    # activation: plain SwiGLU or the GPT-OSS variant with a finite alpha and a limit > 0 (inf allowed)
+    G = moe.MOE_ACT_GPTOSS
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=1.702, act_limit=7.0)) == 0
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=1.0, act_limit=float("inf"))) == 0
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=2)) == 1
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=float("nan"), act_limit=7.0)) == 1
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=1.0, act_limit=0.0)) == 1
+    assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=1.0, act_limit=float("nan"))) == 1
 
 
 def test_workspace_bytes_covers_intermediates():

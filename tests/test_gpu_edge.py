@@ -17,8 +17,9 @@ pytestmark = pytest.mark.gpu
 BF16 = torch.bfloat16
 
 
-def _check_full(inp, tol=TOL_BF16):
-    run = run_stages(inp)
+def _check_full(inp, tol=TOL_BF16, act=None):
+    act = act or (moe.MOE_ACT_SWIGLU, 1.0, float("inf"))
+    run = run_stages(inp, act)
     assert run.status == 0, moe.status_str(run.status)
     s = inp.shape
     _, idx_ref, w_ref = oracle.route(inp.x, inp.Wr, inp.br, s.k)
@@ -28,7 +29,7 @@ def _check_full(inp, tol=TOL_BF16):
     for a, b in ((run.counts, counts), (run.offsets, offsets), (run.perm, perm), (run.inv, inv)):
         assert torch.equal(a.cpu(), b)
     _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, return_exact=True,
-                                 W1_scales=inp.W1_scales, W2_scales=inp.W2_scales)
+                                 W1_scales=inp.W1_scales, W2_scales=inp.W2_scales, act=act)
     assert_close_rms(run.y, y_ref, tol)
     return run
 
@@ -74,6 +75,20 @@ def test_mxfp4_hot_expert_several_passes():
     inp = dataclasses.replace(base, shape=shape, x=x, br=br).to("cuda")
     run = _check_full(inp, TOL_MXFP4)
     assert int(run.counts.max()) > 64
+
+
+@pytest.mark.parametrize("T,D,E,k,I,wfmt", [
+    (512, 256, 8, 2, 512, "bf16"),   # single-SM tcgen05 GEMM tiles
+    (4200, 128, 4, 2, 192, "bf16"),  # SM-pair GEMM tiles
+    (40, 192, 8, 2, 320, "mxfp4"),   # MXFP4 weight-streaming kernels
+    (600, 128, 4, 2, 128, "mxfp4"),  # MXFP4 expanded to bf16, then the GEMM
+])
+def test_gptoss_activation(T, D, E, k, I, wfmt):
+    # the GPT-OSS SwiGLU variant in every mlp1 epilogue; a small limit so that
+    # both clamps act on a good share of the elements
+    act = (moe.MOE_ACT_GPTOSS, 1.702, 0.25)
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + 3 * E, device="cuda", wfmt=wfmt, reject=oracle.gap_reject())
+    _check_full(inp, TOL_MXFP4 if wfmt == "mxfp4" else TOL_BF16, act=act)
 
 
 def test_empty_experts():

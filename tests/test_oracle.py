@@ -277,3 +277,77 @@ def test_mxfp4_nibble_order_and_scale_blocks():
     v = oracle.dequant_mxfp4(codes, scales)[0]
     assert v[0].item() == 1.0 and v[1].item() == 6.0 and v[32].item() == -1.5 * 0.25
     assert torch.count_nonzero(v).item() == 3
+
+
+# ---- GPT-OSS SwiGLU variant (torchtitan GPT-OSS guide, paragraph on the
+# grouped experts' SwiGLU variant): gate clamped from above at `limit` and
+# multiplied by sigmoid(alpha * gate); up clipped to [-limit, limit], plus 1.
+
+def _one_expert_case(T=8, D=32, I=16, seed=21, x_scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = bf16(torch.randn(T, D, generator=g) * x_scale)
+    W1 = bf16(torch.randn(1, 2 * I, D, generator=g) * 0.2)
+    W2 = bf16(torch.randn(1, D, I, generator=g) * 0.2)
+    # biases on a 2^-6 grid in [-1/4, 1/4]: b1 + 1 is exact in bf16
+    b1 = bf16(torch.randint(-16, 17, (1, 2 * I), generator=g).float() / 64)
+    b2 = bf16(torch.randint(-16, 17, (1, D), generator=g).float() / 64)
+    idx = torch.zeros(T, 1, dtype=torch.int32)
+    w = torch.ones(T, 1)
+    return x, idx, w, W1, b1, W2, b2
+
+
+def test_gptoss_act_with_unit_alpha_and_no_limit_is_swiglu_with_up_offset():
+    # alpha = 1, limit = inf: gc = g, uc = u, act = silu(g) * (u + 1), i.e. the
+    # plain SwiGLU layer with 1 added to the up half of b1
+    x, idx, w, W1, b1, W2, b2 = _one_expert_case()
+    I = b1.shape[1] // 2
+    b1_up = b1.clone().float()
+    b1_up[:, I:] += 1.0
+    _, y_var = oracle.ffn_tokens(x, idx, w, W1, b1, W2, b2, return_exact=True, act=(oracle.ACT_GPTOSS, 1.0, math.inf))
+    _, y_ref = oracle.ffn_tokens(x, idx, w, W1, bf16(b1_up), W2, b2, return_exact=True)
+    assert torch.equal(bf16(b1_up).float(), b1_up)  # the offset bias is exact
+    rms = y_ref.pow(2).mean().sqrt()
+    assert float((y_var - y_ref).abs().max()) <= 1e-3 * float(rms)
+    # and it is not the plain layer (the +1 is there)
+    _, y_plain = oracle.ffn_tokens(x, idx, w, W1, b1, W2, b2, return_exact=True)
+    assert float((y_var - y_plain).abs().max()) > 0.1 * float(rms)
+
+
+def test_gptoss_act_with_huge_alpha_is_clamped_relu_glu():
+    # alpha -> inf turns sigmoid(alpha * gc) into a step: act = max(gc, 0) * (uc + 1)
+    # (a ReLU-gated GLU), checked against a dense float64 computation
+    limit = 0.75
+    x, idx, w, W1, b1, W2, b2 = _one_expert_case(seed=22)
+    I = b1.shape[1] // 2
+    u = x.double() @ W1[0].double().T + b1[0].double()
+    assert float(u[:, :I].abs().min()) > 1e-4  # alpha * |g| > 100: the sigmoid is 0 or 1 to double precision
+    gc = u[:, :I].clamp(max=limit)
+    uc = u[:, I:].clamp(-limit, limit)
+    h = (gc.clamp(min=0) * (uc + 1)).to(torch.bfloat16).double()
+    y_dense = h @ W2[0].double().T + b2[0].double()
+    _, y = oracle.ffn_tokens(x, idx, w, W1, b1, W2, b2, return_exact=True, act=(oracle.ACT_GPTOSS, 1e6, limit))
+    assert torch.allclose(y, y_dense, rtol=1e-12, atol=1e-12)
+    assert bool((u[:, :I] > limit).any()) and bool((u[:, I:].abs() > limit).any())  # both clamps are exercised
+
+
+def test_gptoss_act_clamps_gate_only_from_above():
+    # W2 = identity, b2 = 0, one expert, k = 1: y is h itself (bf16). Doubling a
+    # token leaves h unchanged wherever the gate is above the limit and the up
+    # value outside [-limit, limit] at both scales; where the gate is below
+    # -limit it is not clamped, so h changes.
+    D = I = 32
+    limit, alpha = 0.5, 1.702
+    x, idx, w, W1, b1, _, _ = _one_expert_case(D=D, I=I, seed=23, x_scale=4.0)
+    b1 = torch.zeros_like(b1)
+    W2 = bf16(torch.eye(D).unsqueeze(0))
+    b2 = torch.zeros(1, D, dtype=torch.bfloat16)
+    act = (oracle.ACT_GPTOSS, alpha, limit)
+    y1 = oracle.ffn_tokens(x, idx, w, W1, b1, W2, b2, act=act).float()
+    y2 = oracle.ffn_tokens(bf16(2 * x.float()), idx, w, W1, b1, W2, b2, act=act).float()
+    u = x.double() @ W1[0].double().T
+    g, up = u[:, :I], u[:, I:]
+    sat = (g > limit) & (up.abs() > limit)  # g > limit and |u| > limit at x, hence at 2x too
+    low = g < -limit
+    assert bool(sat.any()) and bool(low.any())
+    assert torch.equal(y1[sat], y2[sat])
+    assert bool((y1[low] != y2[low]).all())
