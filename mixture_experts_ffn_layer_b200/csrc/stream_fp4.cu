@@ -135,7 +135,10 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto code_full = [&](int s) { return bar0 + 8u * s; };
-  auto code_empty = [&](int s) { return bar0 + 8u * (SC + s); };  // 8 converter warps + the MMA commit
+  // code_empty: the converter warps release a code stage once the MMA that read
+  // its routed rows has completed (seen as the A-ring slot SA stages later
+  // coming free), so the MMA warp commits only to a_empty
+  auto code_empty = [&](int s) { return bar0 + 8u * (SC + s); };
   auto a_conv = [&](int s) { return bar0 + 8u * (2 * SC + s); };
   auto a_empty = [&](int s) { return bar0 + 8u * (2 * SC + SA + s); };
   const uint32_t accf_bar = bar0 + 8u * (2 * SC + 2 * SA), acce_bar = accf_bar + 8u, done_bar = accf_bar + 16u,
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
     *abort_flag = 0;
     for (int s = 0; s < SC; ++s) {
       mbar_init(code_full(s), 1);
-      mbar_init(code_empty(s), C::kConvWarps + 1);
+      mbar_init(code_empty(s), C::kConvWarps);
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(a_conv(s), C::kConvWarps);
@@ -278,7 +281,6 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
             mma_f16_tmem_a_elect(tmem_base + t * kTok, a0 + t * 64 + kk * 8, bd, idesc, (q | kk) != 0 ? 1u : 0u);
         }
         tc_commit_elect(a_empty(as));
-        tc_commit_elect(code_empty(cs));
         if (++as == SA) {
           as = 0;
           aph ^= 1u;
@@ -323,16 +325,23 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int swz = (r >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r / 2) % 4)
 
-    int cs = 0, as = 0;
+    int cs = 0, as = 0, g = 0;  // g: stage count over all passes
     uint32_t cph = 0, aph = 0;
     for (int pass = 0; pass < npass && !failed; ++pass) {
-      for (int q = 0; q < ncode; ++q) {
+      for (int q = 0; q < ncode; ++q, ++g) {
         if (!__all_sync(0xffffffffu, mbar_wait_backoff(code_full(cs), cph, abort_flag, kWaitNs) &&
                                          mbar_wait_backoff(a_empty(as), aph ^ 1u, abort_flag, kWaitNs))) {
           failed = true;
           break;
         }
         tc_fence_after();
+        if (g >= SA && lane == 0) {
+          // A slot `as` free again: the MMA of stage g - SA has completed, so
+          // that stage's code slot (codes read by this warp long ago, routed
+          // rows read by that MMA) may be refilled
+          const int rs = cs - SA < 0 ? cs - SA + SC : cs - SA;
+          mbar_arrive(code_empty(rs));
+        }
         const uint8_t* crow = code_ring + cs * C::kCodeStageBytes + 2 * kTokBox + t * kCodeTile + r * (kCodeK / 2);
         const uint32_t acol = tmem_base + lane_addr + kAcol0 + (as * C::kTiles + t) * 64;
         const int kq = min(kCodeK, p.K - q * kCodeK);
@@ -357,10 +366,7 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(a_conv(as));
-          mbar_arrive(code_empty(cs));
-        }
+        if (lane == 0) mbar_arrive(a_conv(as));
         if (++as == SA) {
           as = 0;
           aph ^= 1u;
@@ -478,7 +484,9 @@ moe_status_t launch_stream(const CUtensorMap& tm, const uint16_t* in, uint16_t* 
                        static_cast<size_t>(C::kTiles) * kRows * 4 + (2 * C::kAStages + 4) * 8;
   int stages = C::kMaxCodeStages;
   auto bytes = [&](int st) { return fixed + static_cast<size_t>(st) * C::kCodeStageBytes + 2 * st * 8; };
-  while (stages > 2 && bytes(stages) > kSmemLimit) --stages;
+  // the code ring must be deeper than the A ring (a code stage is released SA
+  // stages after it was converted)
+  while (stages > C::kAStages + 1 && bytes(stages) > kSmemLimit) --stages;
   if (bytes(stages) > kSmemLimit) return MOE_ERR_UNSUPPORTED;
   StreamParams q = p;
   q.stages = stages;
