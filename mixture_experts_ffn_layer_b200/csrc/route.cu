@@ -14,7 +14,7 @@
 // from HBM; Wr stays L2-resident.
 // With fewer 128-token tiles than SMs (decode batches) the contraction is also
 // split along K across CTAs so that the SMs all stream x: each split writes
-// its fp32 partial logits, and a second kernel (one warp per token) sums the
+// its fp32 partial logits, and a second kernel (one block per token) sums the
 // splits in a fixed order, adds the bias and takes the same top-k / softmax,
 // so the result is deterministic for given sizes.
 #include "common.cuh"
@@ -253,35 +253,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Sum of the K splits' partial logits (split order 0, 1, ...), bias, top-k
-// and softmax over the chosen logits; one warp per token, lanes over experts.
-// Ties go to the lower expert index, as in the fused epilogue.
-__global__ void __launch_bounds__(128) route_reduce_topk_kernel(const RouteParams p) {
-  const int t = blockIdx.x * 4 + threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (t >= p.T) return;
+// Sum of the K splits' partial logits, bias, top-k and softmax over the
+// chosen logits; one 256-thread block per token. Thread (e, part) sums the
+// splits part, part + nparts, ... in increasing order, the parts are added
+// in part order (a fixed order: deterministic for given sizes), then warp 0
+// selects the top k with lanes over experts. Ties go to the lower expert
+// index, as in the fused epilogue.
+__global__ void __launch_bounds__(256) route_reduce_topk_kernel(const RouteParams p) {
+  __shared__ float part_sum[256];
+  __shared__ float logit[256];
+  const int t = blockIdx.x;
+  const int ep = (p.E + 31) / 32 * 32;  // experts per part, padded to a warp multiple (<= 256)
+  const int nparts = 256 / ep;
+  const int e = threadIdx.x % ep, part = threadIdx.x / ep;
+  float acc = 0.f;
+  if (part < nparts && e < p.E) {
+    const float* src = p.partial + static_cast<int64_t>(t) * p.n_pad + e;
+    const int64_t stride = static_cast<int64_t>(p.T) * p.n_pad;
+    int sp = part;
+    for (; sp + 3 * nparts < p.ksplit; sp += 4 * nparts) {  // four loads in flight, added in order
+      const float a0 = src[sp * stride], a1 = src[(sp + nparts) * stride];
+      const float a2 = src[(sp + 2 * nparts) * stride], a3 = src[(sp + 3 * nparts) * stride];
+      acc += a0;
+      acc += a1;
+      acc += a2;
+      acc += a3;
+    }
+    for (; sp < p.ksplit; sp += nparts) acc += src[sp * stride];
+  }
+  part_sum[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x < ep) {
+    float l = 0.f;
+    for (int q = 0; q < nparts; ++q) l += part_sum[q * ep + threadIdx.x];
+    logit[threadIdx.x] = threadIdx.x < p.E ? l + bf16_bits_to_float(__ldg(p.br + threadIdx.x)) : -FLT_MAX;
+  }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
   constexpr int kPerLane = 8;  // E <= 256
   float v[kPerLane];
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = -FLT_MAX;
-    if (e < p.E) {
-      // fixed order sp = 0, 1, ...; loads issued eight at a time
-      const float* src = p.partial + static_cast<int64_t>(t) * p.n_pad + e;
-      const int64_t stride = static_cast<int64_t>(p.T) * p.n_pad;
-      float acc = 0.f;
-      int sp = 0;
-      for (; sp + 8 <= p.ksplit; sp += 8) {
-        float part[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) part[u] = src[(sp + u) * stride];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc += part[u];
-      }
-      for (; sp < p.ksplit; ++sp) acc += src[sp * stride];
-      v[i] = acc + bf16_bits_to_float(__ldg(p.br + e));
-    }
-  }
+  for (int i = 0; i < kPerLane; ++i) v[i] = lane + 32 * i < p.E ? logit[lane + 32 * i] : -FLT_MAX;
   uint32_t taken = 0;
   float topv[kMaxK];
   int tope[kMaxK];
@@ -295,10 +308,10 @@ __global__ void __launch_bounds__(128) route_reduce_topk_kernel(const RouteParam
     int be = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
-      const int e = lane + 32 * i;
-      if (e < p.E && !(taken >> i & 1u) && v[i] > bv) {  // strict: lower index wins ties
+      const int ei = lane + 32 * i;
+      if (ei < p.E && !(taken >> i & 1u) && v[i] > bv) {  // strict: lower index wins ties
         bv = v[i];
-        be = e;
+        be = ei;
       }
     }
 #pragma unroll
@@ -381,7 +394,7 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   route_tc_kernel<<<dim3((d.T + BM - 1) / BM, p.ksplit), kThreads, smem, s>>>(tx, tw, p);
-  if (p.ksplit > 1) route_reduce_topk_kernel<<<(d.T + 3) / 4, 128, 0, s>>>(p);
+  if (p.ksplit > 1) route_reduce_topk_kernel<<<d.T, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
