@@ -10,14 +10,17 @@
 //               of code stages, each the 128-row block's codes for 128 K
 //               elements (64-byte swizzle; for mlp1 also the 128 up rows)
 //               plus the 32 routed rows (f16, 128-byte swizzle) for them;
-//   warps 2..   converters, two (mlp2) or four (mlp1) per TMEM lane quarter,
-//               each thread half a weight row of a stage: decode the codes with the hardware
-//               E2M1 -> f16 conversion, times 2^(s_block - s_row) where s_row
-//               is the row's largest block scale (so every value is exact in
-//               f16 and none exceeds 6), and store them to tensor memory;
+//   warps 2..   converters, two (mlp2) or four (mlp1) per TMEM lane
+//               quarter, each thread half a weight row of a stage: decode the
+//               codes with the hardware E2M1 -> f16 conversion, times
+//               2^(s_block - s_row) where s_row is the row's largest block
+//               scale (so every value is exact in f16 and none exceeds 6),
+//               and store them to tensor memory;
 //   warp 1      tcgen05.mma with A read from tensor memory (M = 128 weight
 //               rows, K = 16) and B the routed rows from shared memory
-//               (N = 32), into one TMEM accumulator per block (gate, up);
+//               (N = 32), into one TMEM accumulator per block (gate, up),
+//               issued by the whole warp with one lane elected (operands
+//               warp-uniform) and one commit per stage;
 //   warps 2..5  epilogue: TMEM lane = output column; multiply back
 //               2^(s_row - 127), add the bias, SwiGLU (mlp1) or gate weight
 //               (mlp2); for each routed row the 32 lanes of a warp store 32
