@@ -10,7 +10,7 @@ import torch
 import mixture_experts_ffn_layer_b200 as moe
 import oracle
 import synthetic
-from helpers import TOL_BF16, TOL_MXFP4, assert_close_rms, run_stages
+from helpers import TOL_BF16, TOL_MXFP4, assert_close_rms, run_forward, run_stages
 
 pytestmark = pytest.mark.gpu
 
@@ -89,6 +89,19 @@ def test_gptoss_activation(T, D, E, k, I, wfmt):
     act = (moe.MOE_ACT_GPTOSS, 1.702, 0.25)
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + 3 * E, device="cuda", wfmt=wfmt, reject=oracle.gap_reject())
     _check_full(inp, TOL_MXFP4 if wfmt == "mxfp4" else TOL_BF16, act=act)
+
+
+@pytest.mark.parametrize("T,D,E,k,I", [(600, 128, 4, 2, 128), (1024, 256, 8, 4, 192)])
+def test_forward_mxfp4_prefill_matches_stages(T, D, E, k, I):
+    # prefill-sized MXFP4 (weights expanded to bf16 in the workspace): the
+    # one-call path is bitwise the staged path, call after call
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", wfmt="mxfp4", reject=oracle.gap_reject())
+    run = run_stages(inp)
+    assert run.status == 0
+    y1 = run_forward(inp)
+    y2 = run_forward(inp)
+    assert torch.equal(y1.view(torch.int16), run.y.view(torch.int16))
+    assert torch.equal(y2.view(torch.int16), y1.view(torch.int16))
 
 
 def test_empty_experts():
