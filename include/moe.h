@@ -108,7 +108,9 @@ MOE_API moe_status_t moe_check_dims(moe_dims_t d);
  *   -> topk_idx (T,k) int32, ordered by (logit desc, expert asc);
  *      topk_w (T,k) fp32, softmax of the chosen logits (sums to 1).
  * Logits are accumulated in fp32 from the bf16 products (tcgen05 tensor
- * cores, one 128-token tile per CTA); ws holds only the status word. */
+ * cores, one 128-token tile per CTA; batches of at most 18 tiles also split
+ * the reduction over D across CTAs and sum the fp32 partials in a fixed
+ * order, kept in ws). Deterministic for given sizes. */
 MOE_API moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
