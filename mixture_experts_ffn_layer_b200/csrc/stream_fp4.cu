@@ -10,18 +10,19 @@
 //               of code stages, each the 128-row block's codes for 128 K
 //               elements (64-byte swizzle; for mlp1 also the 128 up rows)
 //               plus the 32 routed rows (f16, 128-byte swizzle) for them;
-//   warps 2..   converters, two (mlp2) or four (mlp1) per TMEM lane
+//   warps 5..   converters, two (mlp2) or four (mlp1) per TMEM lane
 //               quarter, each thread half a weight row of a stage: decode the
 //               codes with the hardware E2M1 -> f16 conversion, times
 //               2^(s_block - s_row) where s_row is the row's largest block
 //               scale (so every value is exact in f16 and none exceeds 6),
 //               and store them to tensor memory;
-//   warp 1      tcgen05.mma with A read from tensor memory (M = 128 weight
+//   warps 1..4  tcgen05.mma with A read from tensor memory (M = 128 weight
 //               rows, K = 16) and B the routed rows from shared memory
-//               (N = 32), into one TMEM accumulator per block (gate, up),
-//               issued by the whole warp with one lane elected (operands
-//               warp-uniform) and one commit per stage;
-//   warps 2..5  epilogue: TMEM lane = output column; multiply back
+//               (N = 32); four issuers with an accumulator each (a commit
+//               stalls only its own issuer's MMA stream), each warp-wide with
+//               one lane elected (operands warp-uniform), one commit per stage;
+//   first four converter warps, epilogue: TMEM lane = output column; add the
+//               partial accumulators, multiply back
 //               2^(s_row - 127), add the bias, SwiGLU (mlp1) or gate weight
 //               (mlp2); for each routed row the 32 lanes of a warp store 32
 //               consecutive outputs.
@@ -49,7 +50,9 @@ constexpr int kCodeK = 128;                         // K elements per code stage
 constexpr uint32_t kCodeTile = kRows * kCodeK / 2;  // 8 KB of codes per 128-row block (64-byte swizzle)
 constexpr uint32_t kTokBox = kTok * 64 * 2;         // 64 K of f16 routed rows (128-byte swizzle)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcol0 = 64;                     // TMEM columns [0, 64): accumulators; then the A ring
+constexpr int kMmaWarps = 4;                        // MMA issuers, one accumulator each
+constexpr int kConv0 = 1 + kMmaWarps;               // first converter warp
+constexpr uint32_t kAcol0 = kMmaWarps * kTok;       // TMEM columns [0, 128): accumulators; then the A ring
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -59,9 +62,9 @@ struct Cfg {
   // converter warps, a multiple of four (one group per TMEM lane quarter):
   // mlp1 16 (each thread half a row of one block per stage), mlp2 8 (half a row)
   static constexpr int kConvWarps = kSwiGLU ? 16 : 8;
-  static constexpr int kThreads = (2 + kConvWarps) * 32;
+  static constexpr int kThreads = (kConv0 + kConvWarps) * 32;
   static constexpr int kMaxCodeStages = kSwiGLU ? 8 : 10;
-  static constexpr int kAStages = kSwiGLU ? 3 : 4;  // (512 - 64) / (64 columns per tile)
+  static constexpr int kAStages = kSwiGLU ? 3 : 4;  // (512 - 128) / (64 columns per tile)
   // code stage: [2 routed-row boxes][kTiles code tiles], 1024-byte aligned
   static constexpr uint32_t kCodeStageBytes = 2 * kTokBox + kTiles * kCodeTile;
   static_assert(kAcol0 + kAStages * kTiles * 64 <= kTmemCols, "A ring exceeds tensor memory");
@@ -170,11 +173,11 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(a_conv(s), C::kConvWarps);
-      mbar_init(a_empty(s), 1);
+      mbar_init(a_empty(s), kMmaWarps);
     }
-    mbar_init(accf_bar, 1);
+    mbar_init(accf_bar, kMmaWarps);
     mbar_init(acce_bar, 4);
-    mbar_init(done_bar, 1);
+    mbar_init(done_bar, kMmaWarps);
     mbar_init(sc_bar, 1);
     fence_mbar_init();
   }
@@ -252,9 +255,19 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (whole warp, one lane elected)
+  } else if (warp >= 1 && warp <= kMmaWarps) {
+    // ------------------------------------------------------------ MMA issuers (whole warp, one lane elected)
+    // Four issuing warps, each with its own accumulator and its own commits:
+    // a commit holds up its own warp's MMA stream for a long time, and with
+    // 32 routed rows an MMA is short, so a single issuer would spend most of
+    // each stage waiting. mlp1: issuer m takes tile m / 2 (gate, up) and the
+    // K slices of parity m % 2; mlp2: the K slices kk = m mod 4. The
+    // epilogue adds the partial accumulators in a fixed order.
+    const int m = warp - 1;
+    const int t = kSwiGLU ? m >> 1 : 0;
+    const int kk0 = kSwiGLU ? m & 1 : m, kstep = kSwiGLU ? 2 : 4;
     const uint32_t idesc = idesc_f16_f32(kRows, kTok);
+    const uint32_t dacc = tmem_base + m * kTok;
     int cs = 0, as = 0;
     uint32_t cph = 0, aph = 0;
     bool failed = false;
@@ -272,16 +285,12 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
         }
         tc_fence_after();
         const uint64_t bdesc = desc_kmajor_sw128(smem_u32(code_ring + cs * C::kCodeStageBytes));
-        const uint32_t a0 = tmem_base + kAcol0 + as * C::kTiles * 64;
-        const bool full_stage = p.K - q * kCodeK >= kCodeK;
-#pragma unroll
-        for (int kk = 0; kk < kCodeK / 16; ++kk) {
-          if (kk >= 4 && !full_stage) break;
+        const uint32_t a0 = tmem_base + kAcol0 + (as * C::kTiles + t) * 64;
+        const int nk = p.K - q * kCodeK >= kCodeK ? kCodeK / 16 : 4;  // K is a multiple of 64
+        for (int kk = kk0; kk < nk; kk += kstep) {
           // routed-row box kk / 4, 32-byte K slice kk % 4 (descriptor address field counts 16 bytes)
           const uint64_t bd = bdesc + static_cast<uint64_t>(((kk >> 2) * kTokBox + (kk & 3) * 32) >> 4);
-#pragma unroll
-          for (int t = 0; t < C::kTiles; ++t)
-            mma_f16_tmem_a_elect(tmem_base + t * kTok, a0 + t * 64 + kk * 8, bd, idesc, (q | kk) != 0 ? 1u : 0u);
+          mma_f16_tmem_a_elect(dacc, a0 + kk * 8, bd, idesc, (q != 0 || kk != kk0) ? 1u : 0u);
         }
         tc_commit_elect(a_empty(as));
         if (++as == SA) {
@@ -303,8 +312,8 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
     tc_commit_elect(done_bar);
     mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
   } else {
-    // ------------------------------------------------------------ converters (+ epilogue on warps 2..5)
-    const int cw = warp - 2;    // 0 .. 7
+    // ------------------------------------------------------------ converters (+ epilogue on the first four)
+    const int cw = warp - kConv0;
     const int quarter = warp & 3;  // TMEM lanes this warp may touch: [32 * quarter, 32 * quarter + 32)
     const int r = quarter * 32 + lane;  // weight row within the tile
     // the warps of a lane quarter split a stage: mlp1 (gate | up) x (two K halves), mlp2 two K halves
@@ -379,9 +388,9 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
           cph ^= 1u;
         }
       }
-      if (failed || warp >= 6) continue;
+      if (failed || cw >= 4) continue;
 
-      // ---------------------------------------------------------- epilogue (warps 2..5)
+      // ---------------------------------------------------------- epilogue (the first four converter warps)
       if (!__all_sync(0xffffffffu, mbar_wait_backoff(accf_bar, pass & 1, abort_flag, kWaitNs))) {
         failed = true;
         break;
@@ -400,18 +409,23 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
       const int nb = min(kTok, n_rows - pass * kTok);
 #pragma unroll
       for (int c = 0; c < kTok / 8; ++c) {  // eight routed rows per TMEM load
-        uint32_t vg[8], vu[8];
-        tmem_ld_x8(tmem_base + lane_addr + 8 * c, vg);
-        if (kSwiGLU) tmem_ld_x8(tmem_base + lane_addr + kTok + 8 * c, vu);
+        // the four partial accumulators: mlp1 gate = 0 + 1, up = 2 + 3; mlp2 0 + 1 + 2 + 3
+        uint32_t v0[8], v1[8], v2[8], v3[8];
+        tmem_ld_x8(tmem_base + lane_addr + 0 * kTok + 8 * c, v0);
+        tmem_ld_x8(tmem_base + lane_addr + 1 * kTok + 8 * c, v1);
+        tmem_ld_x8(tmem_base + lane_addr + 2 * kTok + 8 * c, v2);
+        tmem_ld_x8(tmem_base + lane_addr + 3 * kTok + 8 * c, v3);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int jr = 8 * c + i;
           if (!live || jr >= nb) continue;
           const int64_t row = seg0 + pass * kTok + jr;
-          const float g = __uint_as_float(vg[i]) * fg + bg;
+          const float a01 = __uint_as_float(v0[i]) + __uint_as_float(v1[i]);
+          const float a23 = __uint_as_float(v2[i]) + __uint_as_float(v3[i]);
+          const float g = (kSwiGLU ? a01 : a01 + a23) * fg + bg;
           if (kSwiGLU) {
-            const float u = __uint_as_float(vu[i]) * fu + bu;
+            const float u = a23 * fu + bu;
             static_cast<uint16_t*>(p.out)[row * p.n_out + col] = float_to_bf16_bits(glu_act(g, u, p.act));
           } else {
             const int32_t a = p.perm[row];
