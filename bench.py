@@ -50,6 +50,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 7
 
 
+def launches_per_step(T: int, D: int, mxfp4: bool) -> int:
+    """Kernel launches of one staged step: the seven above, plus one per
+    MXFP4 GEMM (weight expansion, or the routed rows' f16 conversion for the
+    weight-streaming kernels), plus the router's partial-logit reduction when
+    it splits K (batches of at most 18 token tiles of 128, D over 64)."""
+    n = LAUNCHES_PER_STEP + (2 if mxfp4 else 0)
+    tiles, kb = -(-T // 128), -(-D // 64)
+    if tiles * 8 <= 148 and min(kb, 148 // tiles) > 1:
+        n += 1
+    return n
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -331,7 +343,7 @@ def run_ours(args):
                            "their own streams, double-buffered, overlapping neighbouring steps' compute"},
             "e2e_serial": {"value": T * world / (e2e_serial_ms / args.steps / 1e3), "unit": UNIT,
                            "how": "same, copy-compute-copy serialised on one stream"},
-            "gpu_launches": (LAUNCHES_PER_STEP + (2 if mx else 0)) * args.steps,
+            "gpu_launches": launches_per_step(T, D, mx) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
