@@ -50,6 +50,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 7
 
 
+def act_tuple(args):
+    """(kind, alpha, limit) of the layer's activation: 0 plain SwiGLU, 1 the GPT-OSS variant."""
+    if getattr(args, "act", "swiglu") == "gptoss":
+        return (1, args.act_alpha, args.act_limit)
+    return (0, 1.0, float("inf"))
+
+
+def act_config(args):
+    return {} if getattr(args, "act", "swiglu") == "swiglu" else {
+        "activation": f"gpt-oss swiglu variant (alpha {args.act_alpha}, limit {args.act_limit})"}
+
+
 def launches_per_step(T: int, D: int, mxfp4: bool) -> int:
     """Kernel launches of one staged step: the seven above, plus one per
     MXFP4 GEMM (weight expansion, or the routed rows' f16 conversion for the
@@ -186,7 +198,7 @@ def run_ours(args):
     T, D, E, k, I = shape.T, shape.D, shape.E, shape.k, shape.I
     R = T * k
     mx = shape.wfmt == "mxfp4"
-    d = moe.dims(T, D, E, k, I, moe.MOE_W_MXFP4 if mx else moe.MOE_W_BF16)
+    d = moe.dims(T, D, E, k, I, moe.MOE_W_MXFP4 if mx else moe.MOE_W_BF16, *act_tuple(args))
     ws = moe.alloc_workspace(d, device=dev)
     i32 = dict(dtype=torch.int32, device=dev)
     topk_idx = torch.empty((T, k), **i32)
@@ -322,7 +334,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not mx:
-        cpu = cpu_baseline(inp, budget_s=args.cpu_budget)
+        cpu = cpu_baseline(inp, budget_s=args.cpu_budget, act=act_tuple(args))
 
     if rank == 0:
         line = {
@@ -331,7 +343,8 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights of the layer shape)",
             "config": {"workload": WORKLOAD_NAMES[workload], "T": T, "D": D, "E": E, "k": k, "I": I,
                        "weights": shape.wfmt, "tokens_per_gpu": T, "parallelism": f"replicas x{world} (token-sharded, "
-                       "no collective)", "l2": f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB per step)"},
+                       "no collective)", "l2": f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB per step)",
+                       **act_config(args)},
             "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peak_tf, "peak_kind": f"{peak_key} ({pk_kind})",
             "stages_ms": stage_ms,
             "roofline": {"kernel": "grouped mlp1 (tcgen05)", "bound": "tensor", "achieved": mlp1_tf, "peak": peak_tf,
@@ -354,13 +367,15 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def cpu_baseline(inp, budget_s=15.0, step_tokens=None):
+def cpu_baseline(inp, budget_s=15.0, step_tokens=None, act=(0, 1.0, float("inf"))):
     """The oracle as it stands, on the host cores, on a bounded token sample."""
     import oracle
 
     x = inp.x.cpu()
     Wr, br = inp.Wr.cpu(), inp.br.cpu()
     W1, b1, W2, b2 = inp.W1.cpu(), inp.b1.cpu(), inp.W2.cpu(), inp.b2.cpu()
+    W1s = None if inp.W1_scales is None else inp.W1_scales.cpu()
+    W2s = None if inp.W2_scales is None else inp.W2_scales.cpu()
     k = inp.shape.k
     T = x.shape[0]
 
@@ -370,7 +385,7 @@ def cpu_baseline(inp, budget_s=15.0, step_tokens=None):
         xs = x[toks].contiguous()
         t0 = time.perf_counter()
         _, idx, w = oracle.route(xs, Wr, br, k)
-        oracle.ffn_tokens(xs, idx, w, W1, b1, W2, b2)
+        oracle.ffn_tokens(xs, idx, w, W1, b1, W2, b2, W1_scales=W1s, W2_scales=W2s, act=act)
         return time.perf_counter() - t0
 
     t1 = run(2, 0)
@@ -401,7 +416,7 @@ def run_reference(args):
         t0 = time.perf_counter()
         _, idx, w = oracle.route(xs, Wr, br, k)
         oracle.ffn_tokens(xs, idx, w, inp.W1, inp.b1, inp.W2, inp.b2, W1_scales=inp.W1_scales,
-                          W2_scales=inp.W2_scales)
+                          W2_scales=inp.W2_scales, act=act_tuple(args))
         return time.perf_counter() - t0
 
     t1 = one(2, 0)
@@ -417,7 +432,7 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": WORKLOAD_NAMES[args.workload], "T": T, "D": shape.D, "E": shape.E, "k": k,
-                   "I": shape.I, "weights": shape.wfmt},
+                   "I": shape.I, "weights": shape.wfmt, **act_config(args)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"{n} of {T} tokens per step (route + FFN + combine per token)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -434,6 +449,10 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOAD_NAMES), default=WORKLOAD,
                     help="the bench line is the 20B shape; the others are for inspection")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--act", choices=["swiglu", "gptoss"], default="swiglu",
+                    help="activation: plain SwiGLU (the benchmark's) or the GPT-OSS variant")
+    ap.add_argument("--act-alpha", type=float, default=1.702, help="GPT-OSS variant: sigmoid slope (caller's choice)")
+    ap.add_argument("--act-limit", type=float, default=7.0, help="GPT-OSS variant: clamp limit (caller's choice)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
     args = ap.parse_args()

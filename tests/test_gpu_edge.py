@@ -53,6 +53,7 @@ def test_shapes(T, D, E, k, I):
     (40, 192, 8, 2, 320),   # three K steps, 2.5 weight blocks per expert
     (1, 128, 32, 4, 64),    # one token
     (96, 256, 24, 1, 192),  # non-power-of-two E
+    (100, 128, 256, 8, 128),  # largest E and k: ~3 rows per expert, some experts empty
 ])
 def test_mxfp4_weight_streaming_shapes(T, D, E, k, I):
     # at most 16 routed rows per expert on average: the MXFP4 weight-streaming kernels
