@@ -333,7 +333,7 @@ def run_ours(args):
     traffic = traffic_from_profile() if workload == WORKLOAD else None
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not mx:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, budget_s=args.cpu_budget, act=act_tuple(args))
 
     if rank == 0:
