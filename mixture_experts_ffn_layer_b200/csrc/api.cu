@@ -202,6 +202,22 @@ moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* per
   const WsLayout L = ws_layout(d);
   uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
   uint16_t* h = at<uint16_t>(ws, L.h);
+  if (stream_fp4_applies(d)) {
+    // MXFP4 weight streaming: x_perm and h are internal here, so the gather
+    // writes the routed rows straight into the f16 form the kernels read and
+    // mlp1 writes h in mlp2's input form (the same values the stage-by-stage
+    // entry points produce with their conversion passes)
+    MOE_REQUIRE(x && aligned32(x) && aligned32(b1) && aligned32(b2) && aligned32(o_perm));
+    MOE_TRY(check_weight(d, W1));
+    MOE_TRY(check_weight(d, W2));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t* tok16 = at<uint16_t>(ws, L.tok16);
+    MOE_TRY(cuda_status(launch_gather(d, x, perm, tok16, status_word(ws), s, true)));
+    MOE_TRY(launch_mlp1_fp4_stream(d, tok16, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h, tok16,
+                                   status_word(ws), s, true, true));
+    return launch_mlp2_fp4_stream(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
+                                  o_perm, tok16, status_word(ws), s, true);
+  }
   MOE_TRY(moe_gather(d, x, perm, x_perm, ws, ws_bytes, stream));
   MOE_TRY(moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, ws_bytes, stream));
   return moe_mlp2(d, h, perm, offsets, topk_w, W2, b2, o_perm, ws, ws_bytes, stream);

@@ -74,8 +74,10 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
                            int chunk = kPermChunk);
+// to_f16: write the gathered rows as f16 (the MXFP4 weight-streaming kernels'
+// input form) instead of bf16.
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
-                          int* status, cudaStream_t s);
+                          int* status, cudaStream_t s, bool to_f16 = false);
 cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32_t* inv, uint16_t* y,
                            int* status, cudaStream_t s);
 
@@ -97,13 +99,17 @@ moe_status_t launch_mlp2_pair(const moe_dims_t& d, const uint16_t* h, const int3
 // are streamed from HBM once and decoded on chip into tcgen05 operands; no
 // expansion pass. Applies when the experts average at most 16 routed rows.
 bool stream_fp4_applies(const moe_dims_t& d);
+// in_f16: x_perm already holds the routed rows in f16 (no conversion pass);
+// h_f16: write h as f16(bf16(h) * 2^-8), the form mlp2's kernel reads.
 moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
                                     const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                                    uint16_t* tok16, int* status, cudaStream_t s);
+                                    uint16_t* tok16, int* status, cudaStream_t s, bool in_f16 = false,
+                                    bool h_f16 = false);
+// in_f16: h already holds f16(bf16(h) * 2^-8) (mlp1 with h_f16).
 moe_status_t launch_mlp2_fp4_stream(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
                                     const int32_t* offsets, const float* topk_w, const uint8_t* codes,
                                     const uint8_t* scales, const uint16_t* b2, float* o_perm, uint16_t* tok16,
-                                    int* status, cudaStream_t s);
+                                    int* status, cudaStream_t s, bool in_f16 = false);
 
 // MXFP4 -> bf16 expansion of an (E, N, K) expert weight (mxfp4.cu).
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t E, int64_t N, int64_t K,

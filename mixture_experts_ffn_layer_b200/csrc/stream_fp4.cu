@@ -35,6 +35,8 @@
 // accumulator is multiplied back. A block whose scale is more than 14 binades
 // below its row's largest one is flushed to zero (its terms are below 2^-14 of
 // the row's scale; a row's scales span a few binades in practice).
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -84,6 +86,7 @@ struct StreamParams {
   void* out;              // h (R, I) bf16 or o_perm (R, D) fp32
   int* status;
   Act act;     // mlp1's activation
+  bool h_f16;  // mlp1: store h as f16(bf16(h) * 2^-8), mlp2's input form, instead of bf16
   int stages;  // pipeline depth that fits shared memory next to the block scales
 };
 
@@ -426,7 +429,9 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
           const float g = (kSwiGLU ? a01 : a01 + a23) * fg + bg;
           if (kSwiGLU) {
             const float u = a23 * fu + bu;
-            static_cast<uint16_t*>(p.out)[row * p.n_out + col] = float_to_bf16_bits(glu_act(g, u, p.act));
+            const uint16_t hb = float_to_bf16_bits(glu_act(g, u, p.act));
+            static_cast<uint16_t*>(p.out)[row * p.n_out + col] =
+                p.h_f16 ? __half_as_ushort(__float2half_rn(bf16_bits_to_float(hb) * (1.0f / 256.0f))) : hb;
           } else {
             const int32_t a = p.perm[row];
             float wgt = 0.f;
@@ -487,14 +492,19 @@ bool make_tmap_codes(CUtensorMap* map, const uint8_t* codes, uint64_t rows, uint
 }
 
 template <bool kSwiGLU>
-moe_status_t launch_stream(const CUtensorMap& tm, const uint16_t* in, uint16_t* in16, const StreamParams& p,
-                           cudaStream_t s) {
+moe_status_t launch_stream(const CUtensorMap& tm, const uint16_t* in, uint16_t* in16, bool in_f16,
+                           const StreamParams& p, cudaStream_t s) {
   using C = Cfg<kSwiGLU>;
-  // routed rows -> f16 (x in_scale) once, then TMA boxes of them are the MMA's B operand
-  const int64_t n8 = p.R * p.K / 8;
-  const int64_t blocks = (n8 + 255) / 256;
-  to_f16_scaled_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(in16), n8, p.in_scale);
+  // routed rows -> f16 (x in_scale) once, then TMA boxes of them are the MMA's
+  // B operand; in_f16: `in` already holds them in that form
+  if (in_f16) {
+    in16 = const_cast<uint16_t*>(in);
+  } else {
+    const int64_t n8 = p.R * p.K / 8;
+    const int64_t blocks = (n8 + 255) / 256;
+    to_f16_scaled_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(in16), n8, p.in_scale);
+  }
   CUtensorMap tt;
   if (!make_tmap_bf16(&tt, in16, p.K, p.R, kTok)) return MOE_ERR_CUDA;
   const size_t fixed = 1024 + 16 + static_cast<size_t>(C::kTiles) * kRows * (p.K / 32) +
@@ -525,7 +535,7 @@ bool stream_fp4_applies(const moe_dims_t& d) {
 
 moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
                                     const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                                    uint16_t* tok16, int* status, cudaStream_t s) {
+                                    uint16_t* tok16, int* status, cudaStream_t s, bool in_f16, bool h_f16) {
   StreamParams p{};
   p.E = d.E;
   p.K = d.D;
@@ -537,17 +547,18 @@ moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm,
   p.bias = b1;
   p.in_scale = 1.0f;
   p.act = act_of(d);
+  p.h_f16 = h_f16;
   p.out = h;
   p.status = status;
   CUtensorMap tm;
   if (!make_tmap_codes(&tm, codes, static_cast<uint64_t>(d.E) * 2 * d.I, d.D / 2)) return MOE_ERR_CUDA;
-  return launch_stream<true>(tm, x_perm, tok16, p, s);
+  return launch_stream<true>(tm, x_perm, tok16, in_f16, p, s);
 }
 
 moe_status_t launch_mlp2_fp4_stream(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
                                     const int32_t* offsets, const float* topk_w, const uint8_t* codes,
                                     const uint8_t* scales, const uint16_t* b2, float* o_perm, uint16_t* tok16,
-                                    int* status, cudaStream_t s) {
+                                    int* status, cudaStream_t s, bool in_f16) {
   StreamParams p{};
   p.E = d.E;
   p.K = d.I;
@@ -564,7 +575,7 @@ moe_status_t launch_mlp2_fp4_stream(const moe_dims_t& d, const uint16_t* h, cons
   p.status = status;
   CUtensorMap tm;
   if (!make_tmap_codes(&tm, codes, static_cast<uint64_t>(d.E) * d.D, d.I / 2)) return MOE_ERR_CUDA;
-  return launch_stream<false>(tm, h, tok16, p, s);
+  return launch_stream<false>(tm, h, tok16, in_f16, p, s);
 }
 
 }  // namespace moe

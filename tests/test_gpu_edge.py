@@ -92,10 +92,14 @@ def test_gptoss_activation(T, D, E, k, I, wfmt):
     _check_full(inp, TOL_MXFP4 if wfmt == "mxfp4" else TOL_BF16, act=act)
 
 
-@pytest.mark.parametrize("T,D,E,k,I", [(600, 128, 4, 2, 128), (1024, 256, 8, 4, 192)])
-def test_forward_mxfp4_prefill_matches_stages(T, D, E, k, I):
-    # prefill-sized MXFP4 (weights expanded to bf16 in the workspace): the
-    # one-call path is bitwise the staged path, call after call
+@pytest.mark.parametrize("T,D,E,k,I", [
+    (600, 128, 4, 2, 128),   # prefill-sized: weights expanded to bf16 in the workspace
+    (1024, 256, 8, 4, 192),
+    (40, 192, 8, 2, 320),    # decode-sized: the one-call path feeds the weight-streaming
+    (64, 2880, 32, 4, 2880),  # kernels f16 rows from the gather and h from mlp1 directly
+])
+def test_forward_mxfp4_matches_stages(T, D, E, k, I):
+    # the one-call MXFP4 path is bitwise the staged path, call after call
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", wfmt="mxfp4", reject=oracle.gap_reject())
     run = run_stages(inp)
     assert run.status == 0
