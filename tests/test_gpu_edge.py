@@ -189,3 +189,29 @@ def test_bounded_wait_times_out_and_reports():
     assert moe.moe_read_device_status(ws) == 0
     inp = synthetic.make_inputs("tiny", device="cuda", reject=oracle.gap_reject())
     assert run_stages(inp).status == 0
+
+
+def _random_shapes(n, seed):
+    g = torch.Generator().manual_seed(seed)
+
+    def ri(lo, hi):
+        return int(torch.randint(lo, hi + 1, (1,), generator=g))
+
+    out = []
+    for i in range(n):
+        E = ri(1, 64)
+        k = ri(1, min(8, E))
+        D, I = 64 * ri(1, 7), 64 * ri(1, 7)
+        T = ri(1, 320)
+        wfmt = "mxfp4" if i % 2 else "bf16"
+        out.append((T, D, E, k, I, wfmt))
+    return out
+
+
+@pytest.mark.parametrize("T,D,E,k,I,wfmt", _random_shapes(10, 2026))
+def test_random_shapes(T, D, E, k, I, wfmt):
+    # seeded random sizes (odd multiples of 64, odd E, k up to 8, ragged T):
+    # every path the sizes select -- single-SM GEMM tiles, MXFP4 expanded or
+    # streamed, the router with or without its K split -- against the oracle
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T * 7 + E, device="cuda", wfmt=wfmt, reject=oracle.gap_reject())
+    _check_full(inp, TOL_MXFP4 if wfmt == "mxfp4" else TOL_BF16)
