@@ -61,8 +61,8 @@ constexpr size_t kSmemLimit = 227 * 1024;
 template <bool kSwiGLU>
 struct Cfg {
   static constexpr int kTiles = kSwiGLU ? 2 : 1;  // gate and up weight blocks for mlp1
-  // converter warps, a multiple of four (one group per TMEM lane quarter):
-  // mlp1 16 (each thread half a row of one block per stage), mlp2 8 (half a row)
+  // converter warps, a multiple of four (one group per TMEM lane quarter);
+  // each thread converts half a weight row of one block per stage
   static constexpr int kConvWarps = kSwiGLU ? 16 : 8;
   static constexpr int kThreads = (kConv0 + kConvWarps) * 32;
   static constexpr int kMaxCodeStages = kSwiGLU ? 8 : 10;
@@ -83,7 +83,7 @@ struct StreamParams {
   float in_scale;         // power of two the routed rows were scaled by in f16
   const int32_t* perm;    // mlp2: gate weight of row r is topk_w[perm[r]]
   const float* topk_w;
-  void* out;              // h (R, I) bf16 or o_perm (R, D) fp32
+  void* out;              // h (R, I) bf16 (f16 with h_f16) or o_perm (R, D) fp32
   int* status;
   Act act;     // mlp1's activation
   bool h_f16;  // mlp1: store h as f16(bf16(h) * 2^-8), mlp2's input form, instead of bf16
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(Cfg<kSwiGLU>::kThreads, 1) stream_fp4_kernel(c
   auto code_full = [&](int s) { return bar0 + 8u * s; };
   // code_empty: the converter warps release a code stage once the MMA that read
   // its routed rows has completed (seen as the A-ring slot SA stages later
-  // coming free), so the MMA warp commits only to a_empty
+  // coming free), so the MMA warps commit only to a_empty
   auto code_empty = [&](int s) { return bar0 + 8u * (SC + s); };
   auto a_conv = [&](int s) { return bar0 + 8u * (2 * SC + s); };
   auto a_empty = [&](int s) { return bar0 + 8u * (2 * SC + SA + s); };
