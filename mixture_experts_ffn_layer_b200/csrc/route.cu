@@ -29,6 +29,10 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 64, kMaxStages = 12, kThreads = 192, kMaxK = 8;
+// Two warps issue the MMAs, each into its own accumulator (even / odd 16-wide
+// K slices), added in that order by the epilogue: a tcgen05.commit stalls the
+// issuing warp's MMA stream, and with N = E these MMAs are short.
+constexpr int kIssuers = 2;
 constexpr int kABytes = BM * BK * 2;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
@@ -58,7 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * kMaxStages + 2));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
@@ -72,10 +76,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(empty_bar(s), kIssuers);
     }
-    mbar_init(tfull_bar, 1);
-    mbar_init(done_bar, 1);
+    mbar_init(tfull_bar, kIssuers);
+    mbar_init(done_bar, kIssuers);
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
@@ -125,15 +129,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // MMA issuer: one 128 x n_pad accumulator over all of K
+  } else {
+    if (warp <= kIssuers) {
+      // ---- MMA issuers (warps 1, 2): whole warp, one lane elected, operands
+      // warp-uniform; issuer i takes the K slices kk = i, i + 2 of each block
+      const int i = warp - 1;
       const uint32_t idesc = idesc_bf16_f32(BM, p.n_pad);
+      const uint32_t dacc = tmem_base + i * p.n_pad;
       int stage = 0;
       uint32_t phase = 0;
       bool failed = false;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, kWaitNs)) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(stage), phase, abort_flag, kWaitNs))) {
           failed = true;
           break;
         }
@@ -141,25 +148,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_addr = smem_u32(smem + stage * stage_bytes);
         const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16(tmem_base, desc_kmajor_sw128(a_addr + kk * 32), desc_kmajor_sw128(b_addr + kk * 32), idesc,
-                   (kb != kb0 || kk != 0) ? 1u : 0u);
-        tc_commit(empty_bar(stage));
+        for (int kk = i; kk < BK / 16; kk += kIssuers)
+          mma_bf16_elect(dacc, desc_kmajor_sw128(a_addr + kk * 32), desc_kmajor_sw128(b_addr + kk * 32), idesc,
+                         (kb != kb0 || kk != i) ? 1u : 0u);
+        tc_commit_elect(empty_bar(stage));
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (failed) {
-        record_status(p.status, MOE_ERR_TIMEOUT);
-        *abort_flag = 1;
+        if (lane == 0) {
+          record_status(p.status, MOE_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
       } else {
-        tc_commit(tfull_bar);
+        tc_commit_elect(tfull_bar);
       }
-      tc_commit(done_bar);
+      tc_commit_elect(done_bar);
       mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
     }
-  } else {
+    if (warp >= 2) {
     // epilogue: thread = token = TMEM lane
     const int q = warp & 3;
     const int t = t0 + q * 32 + lane;
@@ -170,11 +179,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       float* dst = p.partial + (static_cast<int64_t>(blockIdx.y) * p.T + t) * p.n_pad;
       for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
-        uint32_t v[32];
+        uint32_t v[32], w[32];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (c0 + 8 * j < p.n_pad) tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+          if (c0 + 8 * j < p.n_pad) {
+            tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+            tmem_ld_x8(tbase + p.n_pad + c0 + 8 * j, w + 8 * j);
+          }
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
         if (t < p.T) {
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -193,12 +207,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
-        uint32_t v[32];
-        // up to four 8-column loads in flight per wait (warp-uniform bounds)
+        uint32_t v[32], w[32];
+        // up to four 8-column loads of each accumulator in flight per wait
+        // (warp-uniform bounds); the two are added in issuer order
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (c0 + 8 * j < p.n_pad) tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+          if (c0 + 8 * j < p.n_pad) {
+            tmem_ld_x8(tbase + c0 + 8 * j, v + 8 * j);
+            tmem_ld_x8(tbase + p.n_pad + c0 + 8 * j, w + 8 * j);
+          }
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int e = c0 + i;
@@ -242,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (lane == 0) {
       record_status(p.status, MOE_ERR_TIMEOUT);
       *abort_flag = 1;
+    }
     }
   }
 
@@ -371,7 +392,7 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
   p.k = d.k;
   p.n_pad = (d.E + 15) / 16 * 16;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(p.n_pad)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(kIssuers * p.n_pad)) cols <<= 1;  // one accumulator per issuer
   p.tmem_cols = cols;
   p.br = br;
   p.topk_idx = topk_idx;
