@@ -1,7 +1,7 @@
 // The C ABI of include/moe.h: argument validation, workspace layout, and the
-// enqueueing of the kernels of route.cu, permute.cu, grouped_gemm.cu and
-// mxfp4.cu on the caller's stream. No host synchronisation except in
-// moe_read_device_status.
+// enqueueing of the kernels of route.cu, permute.cu, grouped_gemm.cu,
+// grouped_gemm_pair.cu, stream_fp4.cu and mxfp4.cu on the caller's stream.
+// No host synchronisation except in moe_read_device_status.
 #include <cmath>
 
 #include "common.cuh"
