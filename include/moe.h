@@ -137,8 +137,10 @@ MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* 
  * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile).
  * MXFP4 weights: with T*k <= 16*E (a few rows per expert) the codes are
  * streamed once and decoded on chip into tcgen05 operands (weight-streaming
- * kernel); otherwise they are expanded to bf16 in ws first (exact) and the
- * bf16 GEMM runs. */
+ * kernel, which takes the routed rows in f16: |x| must stay below 65504 and
+ * |h| below 2^24 there, far above what a layer's activations reach);
+ * otherwise they are expanded to bf16 in ws first (exact) and the bf16 GEMM
+ * runs. */
 MOE_API moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
                       const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream);
 
