@@ -51,6 +51,21 @@ def test_check_dims_supported_set():
     assert moe.check_dims(moe.dims(8, 64, 4, 2, 64, act=G, act_alpha=1.0, act_limit=float("nan"))) == 1
 
 
+def test_workspace_bytes_cover_the_decode_paths():
+    # 64 tokens at the 20B shape: the router splits K over 45 CTAs (fp32
+    # partial logits, splits * T * E), and MXFP4 weights take the
+    # weight-streaming path (routed rows in f16) instead of expanding them
+    T, D, E, k, I = 64, 2880, 32, 4, 2880
+    R = T * k
+    base = R * D * (2 + 4) + R * I * 2 + R * 4 * 4
+    splits = 45
+    n = moe.workspace_bytes(moe.dims(T, D, E, k, I))
+    assert base + splits * T * E * 4 <= n <= base + splits * T * E * 4 + 1024 * 1024
+    nq = moe.workspace_bytes(moe.dims(T, D, E, k, I, wfmt=moe.MOE_W_MXFP4))
+    assert nq - n >= R * max(D, I) * 2  # routed rows in f16
+    assert nq - n < 2 * 2880 * 2880  # no expanded weights
+
+
 def test_workspace_bytes_covers_intermediates():
     d = moe.dims(8192, 2880, 32, 4, 2880)
     R = 8192 * 4
