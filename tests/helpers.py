@@ -16,7 +16,7 @@ TOL_MXFP4 = 6e-2
 
 
 @dataclasses.dataclass
-class GpuRun:
+class StageRun:
     topk_idx: torch.Tensor
     topk_w: torch.Tensor
     counts: torch.Tensor
@@ -38,7 +38,7 @@ def dims_of(inp: synthetic.LayerInputs, act=SWIGLU):
     return moe.dims(s.T, s.D, s.E, s.k, s.I, moe.MOE_W_MXFP4 if s.wfmt == "mxfp4" else moe.MOE_W_BF16, *act)
 
 
-def run_stages(inp: synthetic.LayerInputs, act=SWIGLU) -> GpuRun:
+def run_stages(inp: synthetic.LayerInputs, act=SWIGLU) -> StageRun:
     """Every stage through its own C-ABI entry point, intermediates kept."""
     s = inp.shape
     dev = inp.x.device
@@ -63,7 +63,7 @@ def run_stages(inp: synthetic.LayerInputs, act=SWIGLU) -> GpuRun:
     moe.moe_mlp2(d, h, perm, offsets, topk_w, inp.W2, inp.b2, o_perm, ws, W2_scales=inp.W2_scales)
     moe.moe_combine(d, o_perm, inv, y, ws)
     status = moe.moe_read_device_status(ws)
-    return GpuRun(topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, y, status)
+    return StageRun(topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, y, status)
 
 
 def run_forward(inp: synthetic.LayerInputs, act=SWIGLU) -> torch.Tensor:
