@@ -93,6 +93,12 @@ def test_argument_errors_are_synchronous():
     dq = moe.dims(64, 64, 4, 2, 64, wfmt=moe.MOE_W_MXFP4)
     wq = _binding.Weight(1 << 20, None)  # MXFP4 without scales
     assert lib.moe_mlp1(dq, fake, fake, wq, fake, fake, fake, 1 << 30, None) == 1
+    wq_mis = _binding.Weight(1 << 20, (1 << 20) + 16)  # scales not 32-byte aligned
+    assert lib.moe_mlp1(dq, fake, fake, wq_mis, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.moe_mlp2(dq, fake, fake, fake, fake, wq_mis, fake, fake, fake, 1 << 30, None) == 1
+    # the GPT-OSS activation with an invalid limit fails every entry point's dims check
+    dbad = moe.dims(64, 64, 4, 2, 64, act=moe.MOE_ACT_GPTOSS, act_alpha=1.0, act_limit=-1.0)
+    assert lib.moe_mlp1(dbad, fake, fake, _binding.Weight(1 << 20, None), fake, fake, fake, 1 << 30, None) == 1
     assert lib.moe_forward(moe.dims(64, 64, 4, 9, 64), fake, fake, fake, w, fake, w, fake, fake, fake, 0, None) == 1
     assert lib.moe_read_device_status(None, None) == 1
     assert lib.moe_selftest_wait_timeout(None, 1000, None) == 1
