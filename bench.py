@@ -46,8 +46,8 @@ WORKLOAD_NAMES = {
 METRIC = "MoE layer tokens/s and TFLOP/s at 1 B200, % of tensor-core peak"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# kernels per step: route 1, permute 2, gather 1, mlp1 1, mlp2 1, combine 1
-LAUNCHES_PER_STEP = 7
+# kernels per step: route 1, permute 3, gather 1, mlp1 1, mlp2 1, combine 1
+LAUNCHES_PER_STEP = 8
 
 
 def act_tuple(args):
@@ -177,6 +177,51 @@ def step_throughput(elapsed_ms, steps, tokens_per_rank, world):
     tokens_per_rank tokens per step (replicas, weak scaling)."""
     ms = elapsed_ms / steps
     return ms, tokens_per_rank * world / (ms / 1e3)
+
+
+def rooflines(shape, inp, stage_ms, mlp1_ms, peak_tf, pk, pk_kind, workload):
+    """The dominant kernel's roofline against the resource that bounds it, and
+    the memory-bound stages' achieved HBM bandwidth.
+
+    mlp1 (grouped GEMM + SwiGLU) dominates every workload. With few routed rows
+    per expert (T*k <= 16*E, decode-sized MXFP4 batches) it is bound by
+    streaming the expert weights from HBM: algorithmic bytes = W1 (codes and
+    scales, or bf16) + the routed rows read + h written. Otherwise it is bound
+    by the tensor cores: 4*R*D*I FLOP per launch."""
+    T, D, E, k, I = shape.T, shape.D, shape.E, shape.k, shape.I
+    R = T * k
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    w1_bytes = sum(t.numel() * t.element_size() for t in (inp.W1, inp.W1_scales) if t is not None)
+    w2_bytes = sum(t.numel() * t.element_size() for t in (inp.W2, inp.W2_scales) if t is not None)
+    decode = T * k <= 16 * E
+    if decode:
+        mlp1_bytes = w1_bytes + R * D * 2 + R * I * 2
+        ach = mlp1_bytes / (mlp1_ms / 1e3) / 1e9
+        roof = {"kernel": "grouped mlp1 + SwiGLU (tcgen05)", "bound": "hbm", "achieved": ach, "peak": hbm,
+                "unit": "GB/s", "frac": ach / hbm, "traffic": None, "peak_kind": f"hbm_gbs ({pk_kind})",
+                "algorithmic": f"W1 {w1_bytes} B + routed rows {R * D * 2} B + h {R * I * 2} B per launch"}
+    else:
+        mlp1_flops = 4.0 * R * D * I
+        tf = mlp1_flops / (mlp1_ms / 1e3) / 1e12
+        traffic = traffic_from_profile() if workload == WORKLOAD else None
+        roof = {"kernel": "grouped mlp1 + SwiGLU (tcgen05)", "bound": "tensor", "achieved": tf, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": traffic,
+                "algorithmic": f"4*R*D*I = {mlp1_flops:.4g} FLOP per launch"}
+    # memory-bound stages: algorithmic bytes per launch / CUDA-event time
+    mem = {
+        "route": T * D * 2 + E * D * 2 + R * 8,
+        "gather": R * D * 2 * 2,
+        "combine": R * D * 4 + T * D * 2 + R * 4,
+    }
+    if decode:
+        mem["mlp2"] = w2_bytes + R * I * 2 + R * D * 4
+    out = {}
+    for name, nbytes in mem.items():
+        ms = stage_ms.get(name)
+        if ms:
+            gbs = nbytes / (ms / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "bytes": nbytes, "ms": ms, "achieved_gbs": gbs, "frac": gbs / hbm}
+    return roof, out
 
 
 # ------------------------------------------------------------------ our arm
@@ -329,8 +374,11 @@ def run_ours(args):
     peak_tf = float(pk.get(peak_key, FALLBACK_PEAKS[peak_key]))
     mlp1_flops = 4.0 * R * D * I
     wbytes = sum(t.numel() * t.element_size() for t in (inp.W1, inp.W2, inp.W1_scales, inp.W2_scales) if t is not None)
-    mlp1_tf = mlp1_flops / (mlp1_ms / 1e3) / 1e12
-    traffic = traffic_from_profile() if workload == WORKLOAD else None
+    roofline, stage_roofline = rooflines(shape, inp, stage_ms, mlp1_ms, peak_tf, pk, pk_kind, workload)
+    counts_h = counts.cpu().tolist()
+    routing = {"tokens_per_expert": counts_h, "min": min(counts_h), "max": max(counts_h),
+               "experts_le8": sum(c <= 8 for c in counts_h), "experts_gt1000": sum(c > 1000 for c in counts_h),
+               "tile_rows_128": sum(-(-c // 128) * 128 for c in counts_h), "rows": R}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -347,9 +395,9 @@ def run_ours(args):
                        **act_config(args)},
             "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peak_tf, "peak_kind": f"{peak_key} ({pk_kind})",
             "stages_ms": stage_ms,
-            "roofline": {"kernel": "grouped mlp1 (tcgen05)", "bound": "tensor", "achieved": mlp1_tf, "peak": peak_tf,
-                         "unit": "TFLOP/s", "frac": mlp1_tf / peak_tf, "traffic": traffic,
-                         "algorithmic": f"4*R*D*I = {mlp1_flops:.4g} FLOP per launch"},
+            "roofline": roofline,
+            "stage_rooflines": stage_roofline,
+            "routing": routing,
             "e2e": {"value": T * world / (e2e_ms / args.steps / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2,
                     "how": "moe_forward per step with its x H2D and y D2H copies in the timed region; copies on "

@@ -104,6 +104,10 @@ MOE_API size_t moe_workspace_bytes(moe_dims_t d);
 MOE_API moe_status_t moe_check_dims(moe_dims_t d);
 
 /* Router linear + top-k + softmax over the chosen logits.
+ * Defined by: torchtitan GPT-OSS guide, "HuggingFace weight adapter" (the
+ * router is a linear layer with weight and bias, one logit per expert);
+ * from-scratch GPT-OSS write-up, "model flow" (expert routing, top-4 of 32
+ * experts); the softmax is taken over the k chosen logits only.
  *   x (T,D) bf16, Wr (E,D) bf16, br (E) bf16
  *   -> topk_idx (T,k) int32, ordered by (logit desc, expert asc);
  *      topk_w (T,k) fp32, softmax of the chosen logits (sums to 1).
@@ -115,6 +119,9 @@ MOE_API moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* 
                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
 /* Group the R = T*k assignments a = t*k + j by expert (stable in a).
+ * Defined by: torchtitan GPT-OSS guide, "grouped matrix multiplication"
+ * (tokens sorted by expert, num_tokens_per_expert, offsets = cumsum of it,
+ * computed without a device-to-host sync).
  *   topk_idx (T,k) int32
  *   -> counts (E) int32 tokens per expert; offsets (E+1) int32 exclusive
  *      prefix sums (offsets[0] = 0, offsets[E] = R); perm (R) int32, row r of
@@ -125,11 +132,18 @@ MOE_API moe_status_t moe_route(moe_dims_t d, const uint16_t* x, const uint16_t* 
 MOE_API moe_status_t moe_permute(moe_dims_t d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                          int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream);
 
-/* Gather the routed rows: x_perm[r] = x[perm[r] / k], x_perm (R,D) bf16. */
+/* Gather the routed rows: x_perm[r] = x[perm[r] / k], x_perm (R,D) bf16.
+ * Defined by: torchtitan GPT-OSS guide, "grouped matrix multiplication"
+ * (the grouped GEMM's input is the token rows in expert-sorted order). */
 MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
                         void* ws, size_t ws_bytes, void* stream);
 
-/* Grouped mlp1 + bias + SwiGLU over the expert segments of x_perm:
+/* Grouped mlp1 + bias + SwiGLU over the expert segments of x_perm.
+ * Defined by: torchtitan GPT-OSS guide, "grouped matrix multiplication"
+ * (mlp1 as one grouped GEMM over the expert segments given by offsets,
+ * weights stored (num_experts, out_dim, in_dim) with a per-expert bias,
+ * then the SwiGLU; the guide's GPT-OSS variant is moe_act_t's second
+ * form) and "expert-parallel sharding" (mlp1 weight E x 2I x D, bias E x 2I).
  * for r in [offsets[e], offsets[e+1]):
  *   u = W1[e] . x_perm[r] + b1[e] (fp32 accumulate), h[r,i] = bf16(act(u[i], u[I+i]))
  *   with act = d.act (plain SwiGLU or the GPT-OSS variant, see moe_act_t).
@@ -144,7 +158,11 @@ MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* 
 MOE_API moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
                       const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream);
 
-/* Grouped mlp2 + bias + gate weight over the expert segments of h:
+/* Grouped mlp2 + bias + gate weight over the expert segments of h.
+ * Defined by: torchtitan GPT-OSS guide, "grouped matrix multiplication"
+ * (mlp2 as the second grouped GEMM, weights E x D x I with bias E x D) and
+ * the write-up's "weighted combination" (each expert output scaled by its
+ * routing weight; here inside mlp2's epilogue).
  *   o_perm[r] = topk_w[perm[r]] * (W2[e] . h[r] + b2[e]), stored fp32.
  *   h (R,I) bf16, perm (R), offsets (E+1), topk_w (T*k) fp32, W2 (E,D,I),
  *   b2 (E,D) bf16 -> o_perm (R,D) fp32. The expert outputs stay fp32 so that
@@ -153,13 +171,17 @@ MOE_API moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* pe
                       const float* topk_w, moe_weight_t W2, const uint16_t* b2, float* o_perm,
                       void* ws, size_t ws_bytes, void* stream);
 
-/* The expert FFN of all routed rows: moe_gather, moe_mlp1, moe_mlp2 with the
+/* Defined by: torchtitan GPT-OSS guide, "grouped matrix multiplication" (the
+ * whole grouped-experts forward: gather, mlp1 + SwiGLU, mlp2).
+ * The expert FFN of all routed rows: moe_gather, moe_mlp1, moe_mlp2 with the
  * gathered rows and h kept in ws. o_perm (R,D) fp32 as moe_mlp2. */
 MOE_API moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* perm, const int32_t* offsets,
                              const float* topk_w, moe_weight_t W1, const uint16_t* b1, moe_weight_t W2,
                              const uint16_t* b2, float* o_perm, void* ws, size_t ws_bytes, void* stream);
 
-/* Weighted combine back to token order (the gate weight is already applied):
+/* Weighted combine back to token order (the gate weight is already applied).
+ * Defined by: from-scratch GPT-OSS write-up, "model flow" (weighted
+ * combination of the top-4 expert outputs per token).
  *   y[t] = bf16( sum_{j<k} o_perm[inv[t*k+j]] ), o_perm (R,D) fp32, summed in
  *   fp32 in j order. A gather: each output row is written once, no atomics,
  *   bitwise deterministic. */
@@ -167,6 +189,8 @@ MOE_API moe_status_t moe_combine(moe_dims_t d, const float* o_perm, const int32_
                          void* ws, size_t ws_bytes, void* stream);
 
 /* The whole layer in one call: route, permute, gather, mlp1, mlp2, combine,
+ * as the write-up's "model flow" (routing, expert compute, weighted
+ * combination) and the torchtitan guide's grouped-experts forward define it;
  * enqueued on `stream` with every intermediate in ws.
  *   x (T,D) bf16, Wr (E,D), br (E), W1/b1, W2/b2 as above -> y (T,D) bf16. */
 MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,

@@ -3,12 +3,14 @@
 // The torchtitan GPT-OSS guide ("grouped matrix multiplication") feeds the
 // grouped GEMMs with rows sorted by expert and offsets = cumsum of
 // num_tokens_per_expert, computed without a device-to-host sync. Here the
-// R = T*k assignments a = t*k + j are sorted stably by expert in two launches:
+// R = T*k assignments a = t*k + j are sorted stably by expert in three launches:
 //   1. per-block histograms of `chunk` assignments (shared-memory counters);
-//   2. each block derives its per-expert base from the histograms of the
-//      blocks before it plus the exclusive scan over experts, then ranks its
-//      assignments in order with warp match/popc and per-warp counts -- the
-//      position of every assignment is fixed by (expert, a), never by atomics.
+//   2. a column scan per expert turns the histograms into per-block prefixes
+//      and per-expert totals (counts);
+//   3. each block takes its per-expert base from its prefix plus the
+//      exclusive scan of the totals over experts, then ranks its assignments
+//      in order with warp match/popc and per-warp counts -- the position of
+//      every assignment is fixed by (expert, a), never by atomics.
 // The combine (from-scratch GPT-OSS write-up, "weighted combination") is a
 // gather: every output row sums its k expert rows in slot order.
 #include "common.cuh"
@@ -36,41 +38,75 @@ __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* 
   for (int e = threadIdx.x; e < E; e += blockDim.x) block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
 }
 
+// Column scan of the block histograms, one CTA per expert e: block_counts[b][e]
+// becomes the number of assignments to e in blocks before b (exclusive prefix
+// over blocks, in place), and counts[e] the total.
+__global__ void __launch_bounds__(kPermThreads) perm_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E,
+                                                                 int32_t* __restrict__ counts) {
+  constexpr int kWarps = kPermThreads / 32;
+  __shared__ int wsum[kWarps];
+  const int e = blockIdx.x, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  int carry = 0;
+  for (int b0 = 0; b0 < nblk; b0 += kPermThreads) {
+    const int b = b0 + tid;
+    const int v = b < nblk ? block_counts[static_cast<int64_t>(b) * E + e] : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += u;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int ws = wsum[w];
+      if (w < warp) before += ws;
+      total += ws;
+    }
+    if (b < nblk) block_counts[static_cast<int64_t>(b) * E + e] = carry + before + incl - v;
+    carry += total;
+    __syncthreads();
+  }
+  if (tid == 0) counts[e] = carry;
+}
+
 __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
-                                                                    int chunk, const int32_t* __restrict__ block_counts,
-                                                                    int32_t* __restrict__ counts,
+                                                                    int chunk, const int32_t* __restrict__ block_pre,
+                                                                    const int32_t* __restrict__ counts,
                                                                     int32_t* __restrict__ offsets,
                                                                     int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   constexpr int kWarps = kPermThreads / 32;
-  __shared__ int tot[256];
   __shared__ int base[256];
   __shared__ int wcnt[kWarps][256];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int nblk = gridDim.x, blk = blockIdx.x;
+  const int blk = blockIdx.x;
 
-  // Per-expert totals and this block's prefix over the blocks before it.
-  int pre = 0;
-  if (tid < E) {
-    int total = 0;
-    for (int b = 0; b < nblk; ++b) {
-      int c = block_counts[static_cast<int64_t>(b) * E + tid];
-      if (b < blk) pre += c;
-      total += c;
+  // Expert offsets (exclusive scan of the totals over experts, E <= 256 =
+  // the block size) plus this block's prefix over the blocks before it.
+  {
+    const int c = tid < E ? counts[tid] : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += u;
     }
-    tot[tid] = total;
-  }
-  __syncthreads();
-  if (tid < E) {
-    int off = 0;
-    for (int e = 0; e < tid; ++e) off += tot[e];
-    base[tid] = off + pre;
-    if (blk == 0) {
-      counts[tid] = tot[tid];
-      offsets[tid] = off;
-      if (tid == E - 1) offsets[E] = off + tot[tid];
+    if (lane == 31) wcnt[0][warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wcnt[0][w];
+    const int off = before + incl - c;
+    if (tid < E) {
+      base[tid] = off + block_pre[static_cast<int64_t>(blk) * E + tid];
+      if (blk == 0) {
+        offsets[tid] = off;
+        if (tid == E - 1) offsets[E] = off + c;
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
 
   const int64_t a0 = static_cast<int64_t>(blk) * chunk;
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -170,6 +206,7 @@ cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
   const int nblk = static_cast<int>((R + chunk - 1) / chunk);
   perm_hist_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, chunk, block_counts, status);
+  perm_scan_kernel<<<d.E, kPermThreads, 0, s>>>(block_counts, nblk, d.E, counts);
   perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, chunk, block_counts, counts, offsets, perm,
                                                     inv);
   return cudaGetLastError();
@@ -209,6 +246,8 @@ cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32
 // (the histogram kernel writes all of its block's counts, so nothing has to
 // start at zero), and two calls whose kernels overlap on the GPU -- on two
 // streams, or on two host threads -- race on it.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 namespace moe {
@@ -221,21 +260,58 @@ __device__ __align__(256) int32_t g_noalloc_block_counts[kNoAllocScratchInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-int32_t* g_noalloc_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // the CUDA context the address belongs to (0 = none yet)
+  int32_t* ptr;
+};
+ScratchAddr g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device. The host-side
-// name of a __device__ array is only a stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// Unique id of the calling thread's current CUDA context (cuCtxGetId: never
+// reused within the process), fetched through the runtime's driver entry
+// point query so the library needs no libcuda link.
+bool current_ctx_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || !a)
+      return false;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess || !b)
+      return false;
+    get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+    get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current device's context. The
+// host-side name of a __device__ array is only a stand-in, so the address is
+// looked up with the device current, once per context, and cached. A new
+// context on the device (after cudaDeviceReset, for instance, the module is
+// loaded again and the array may move) has a new id and gets a new lookup.
 moe_status_t noalloc_scratch(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  unsigned long long id = 0;
+  const bool have_ctx = current_ctx_id(&id) && id != 0;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  ScratchAddr& a = g_noalloc_addr[dev];
+  if (!have_ctx || a.ctx_id != id || !a.ptr) {
+    // the lookup also binds the device's primary context to this thread if
+    // no runtime call has done so yet
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_block_counts) != cudaSuccess || !p) return MOE_ERR_CUDA;
-    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+    if (!current_ctx_id(&id) || id == 0) return MOE_ERR_CUDA;
+    a.ptr = static_cast<int32_t*>(p);
+    a.ctx_id = id;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return MOE_OK;
 }
 

@@ -78,30 +78,81 @@ def test_workspace_bytes_covers_intermediates():
         moe.workspace_bytes(moe.dims(8, 64, 4, 5, 64))
 
 
+class _Arena:
+    """Addresses for the argument-error tests. On a machine with a GPU every
+    address lies inside one real device buffer large enough for the tiny
+    layer below (so even a check that regressed could only touch memory that
+    exists); on a machine without one no kernel can run at all, and plain
+    integers stand in for device addresses."""
+
+    def __init__(self, size=32 << 20):
+        import torch
+
+        self.SIZE = size
+        if torch.cuda.is_available():
+            self.buf = torch.zeros(self.SIZE, dtype=torch.uint8, device="cuda")
+            self.base = self.buf.data_ptr()
+        else:
+            self.buf = None
+            self.base = 1 << 32
+        self.next = 0
+
+    def take(self, nbytes=1 << 20):
+        """A 256-byte aligned address with `nbytes` of the buffer behind it."""
+        at = self.next
+        self.next += (nbytes + 255) // 256 * 256
+        assert self.next <= self.SIZE
+        return self.base + at
+
+
 def test_argument_errors_are_synchronous():
     lib = moe.load()
     d = moe.dims(64, 64, 4, 2, 64)
+    ar = _Arena()
     vp = ctypes.c_void_p
-    fake = vp(1 << 20)  # never dereferenced: validation fails first
-    assert lib.moe_route(d, None, fake, fake, fake, fake, fake, 1 << 30, None) == 1
-    assert lib.moe_route(d, vp((1 << 20) + 8), fake, fake, fake, fake, fake, 1 << 30, None) == 1  # misaligned x
-    assert lib.moe_route(d, fake, fake, fake, fake, fake, fake, 16, None) == 3
-    assert lib.moe_permute(d, fake, fake, fake, fake, fake, fake, 16, None) == 3  # workspace too small
-    assert lib.moe_permute(d, fake, fake, fake, fake, fake, vp((1 << 20) + 4), 1 << 30, None) == 1
+    ws_n = moe.workspace_bytes(d)
+    ws = vp(ar.take(ws_n))
+    p = [vp(ar.take()) for _ in range(8)]  # each 1 MB: more than any tensor of this layer
+    mis8 = vp(ar.take() + 8)  # inside the buffer, not 32-byte aligned
+    assert lib.moe_route(d, None, p[0], p[1], p[2], p[3], ws, ws_n, None) == 1
+    assert lib.moe_route(d, mis8, p[0], p[1], p[2], p[3], ws, ws_n, None) == 1  # misaligned x
+    assert lib.moe_route(d, p[0], p[1], p[2], p[3], p[4], ws, 16, None) == 3  # workspace too small
+    assert lib.moe_permute(d, p[0], p[1], p[2], p[3], p[4], ws, 16, None) == 3
+    assert lib.moe_permute(d, p[0], p[1], p[2], p[3], p[4], vp(ar.take() + 4), ws_n, None) == 1  # misaligned ws
     w = _binding.Weight(None, None)
-    assert lib.moe_mlp1(d, fake, fake, w, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.moe_mlp1(d, p[0], p[1], w, p[2], p[3], ws, ws_n, None) == 1
     dq = moe.dims(64, 64, 4, 2, 64, wfmt=moe.MOE_W_MXFP4)
-    wq = _binding.Weight(1 << 20, None)  # MXFP4 without scales
-    assert lib.moe_mlp1(dq, fake, fake, wq, fake, fake, fake, 1 << 30, None) == 1
-    wq_mis = _binding.Weight(1 << 20, (1 << 20) + 16)  # scales not 32-byte aligned
-    assert lib.moe_mlp1(dq, fake, fake, wq_mis, fake, fake, fake, 1 << 30, None) == 1
-    assert lib.moe_mlp2(dq, fake, fake, fake, fake, wq_mis, fake, fake, fake, 1 << 30, None) == 1
+    wsq_n = moe.workspace_bytes(dq)
+    wsq = vp(ar.take(wsq_n))
+    wq = _binding.Weight(p[5].value, None)  # MXFP4 without scales
+    assert lib.moe_mlp1(dq, p[0], p[1], wq, p[2], p[3], wsq, wsq_n, None) == 1
+    wq_mis = _binding.Weight(p[5].value, p[6].value + 16)  # scales not 32-byte aligned
+    assert lib.moe_mlp1(dq, p[0], p[1], wq_mis, p[2], p[3], wsq, wsq_n, None) == 1
+    assert lib.moe_mlp2(dq, p[0], p[1], p[2], p[3], wq_mis, p[4], p[7], wsq, wsq_n, None) == 1
     # the GPT-OSS activation with an invalid limit fails every entry point's dims check
     dbad = moe.dims(64, 64, 4, 2, 64, act=moe.MOE_ACT_GPTOSS, act_alpha=1.0, act_limit=-1.0)
-    assert lib.moe_mlp1(dbad, fake, fake, _binding.Weight(1 << 20, None), fake, fake, fake, 1 << 30, None) == 1
-    assert lib.moe_forward(moe.dims(64, 64, 4, 9, 64), fake, fake, fake, w, fake, w, fake, fake, fake, 0, None) == 1
+    assert lib.moe_mlp1(dbad, p[0], p[1], _binding.Weight(p[5].value, None), p[2], p[3], ws, ws_n, None) == 1
+    assert lib.moe_forward(moe.dims(64, 64, 4, 9, 64), p[0], p[1], p[2], w, p[3], w, p[4], p[5], ws, 0, None) == 1
     assert lib.moe_read_device_status(None, None) == 1
     assert lib.moe_selftest_wait_timeout(None, 1000, None) == 1
-    assert lib.moe_selftest_wait_timeout(fake, 0, None) == 1
-    assert lib.moe_selftest_wait_timeout(fake, 3_000_000_000, None) == 1
+    assert lib.moe_selftest_wait_timeout(ws, 0, None) == 1
+    assert lib.moe_selftest_wait_timeout(ws, 3_000_000_000, None) == 1
     assert moe.status_str(6) == "device: index or offset out of range"
+
+
+def test_noalloc_permute_size_limit_boundary():
+    # The workspace-free permutation keeps one int32 per (block of 2048
+    # assignments, expert) in a fixed 65536-entry array: exactly 65536 entries
+    # are accepted (checked on the GPU against the oracle in its own test
+    # file), one block more is refused before anything is enqueued.
+    lib = moe.load()
+    ar = _Arena(80 << 20)  # the largest case's perm array is 67 MB
+    vp = ctypes.c_void_p
+    for T, E, k in [(256 * 2048 + 1, 256, 1), (2048 * 2048 + 1, 32, 1), (8192 * 2048 // 4 + 1, 8, 4)]:
+        blocks = -(-(T * k) // 2048)
+        assert blocks * E == 65536 + E
+        d = moe.dims(T, 64, E, k, 64)
+        assert lib.moe_permute_noalloc(d, *[vp(ar.base)] * 5, None) == 2
+    # invalid dims are refused by the dims check first
+    assert lib.moe_permute_noalloc(moe.dims(8, 64, 4, 5, 64), *[vp(ar.base)] * 5, None) == 1
+    assert lib.moe_permute_noalloc(moe.dims(8, 64, 4, 2, 64), None, *[vp(ar.base)] * 4, None) == 1

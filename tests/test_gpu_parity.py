@@ -70,16 +70,31 @@ def test_large_shapes_reduced_tokens(name, T, n):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,n", [("gptoss20b", 64), ("gptoss120b_zipf", 64)])
-def test_full_size_sampled(name, n):
+@pytest.mark.parametrize("name", ["gptoss20b", "gptoss120b_zipf", "gptoss20b_mxfp4"])
+def test_full_size_sampled(name):
+    # Every graded full-size workload, in the launch configuration the
+    # benchmark times: routing, counts, offsets, perm, inv and the gathered rows
+    # are compared on all tokens; the layer output on 2048 seeded random
+    # tokens plus every token routed to an expert with fewer than 64 rows
+    # (tokens are independent, so a sample checks the same arithmetic; with
+    # ~1024 rows per expert it reaches every 128-row tile of most experts).
     inp = _inputs(name)
     run = run_stages(inp)
     assert run.status == 0
     idx_ref, w_ref = _check_routing(inp, run)
-    toks = sample_tokens(idx_ref, inp.shape.E, n)
+    counts = run.counts.cpu()
+    if name == "gptoss120b_zipf":
+        # the skew the 120B-shaped workload calls for: some experts with 0-8
+        # tokens, others with more than 1000
+        assert int(counts.min()) <= 8 and int(counts.max()) > 1000, counts.tolist()
+    toks = sample_tokens(idx_ref, inp.shape.E, 2048)
+    rare = (counts < 64) & (counts > 0)
+    assert bool(torch.isin(torch.nonzero(rare[idx_ref.long()].any(dim=1)).flatten(), toks).all())
     _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, tokens=toks,
-                                 return_exact=True)
-    assert_close_rms(run.y.cpu()[toks], y_ref, TOL_BF16)
+                                 W1_scales=inp.W1_scales, W2_scales=inp.W2_scales, return_exact=True)
+    tol = TOL_MXFP4 if inp.shape.wfmt == "mxfp4" else TOL_BF16
+    err = assert_close_rms(run.y.cpu()[toks], y_ref, tol)
+    print(f"{name}: {toks.numel()} tokens, max|y - y_ref| / rms = {err:.4g}")
     # the one-call path launches the same kernels
     y = run_forward(inp)
     assert torch.equal(y.view(torch.int16), run.y.view(torch.int16))
