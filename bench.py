@@ -103,7 +103,7 @@ class Clocks:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -210,7 +210,7 @@ def rooflines(shape, inp, stage_ms, mlp1_ms, peak_tf, pk, pk_kind, workload):
     # memory-bound stages: algorithmic bytes per launch / CUDA-event time
     mem = {
         "route": T * D * 2 + E * D * 2 + R * 8,
-        "gather": R * D * 2 * 2,
+        "gather": T * D * 2 + R * D * 2 + R * 4,  # each token row read once (k copies from L2), R rows written
         "combine": R * D * 4 + T * D * 2 + R * 4,
     }
     if decode:

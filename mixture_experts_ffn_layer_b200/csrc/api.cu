@@ -1,6 +1,6 @@
 // The C ABI of include/moe.h: argument validation, workspace layout, and the
 // enqueueing of the kernels of route.cu, permute.cu, grouped_gemm.cu,
-// grouped_gemm_pair.cu, stream_fp4.cu and mxfp4.cu on the caller's stream.
+// grouped_gemm_pair.cu and mx_gemm.cu on the caller's stream.
 // No host synchronisation except in moe_read_device_status.
 #include <cmath>
 
@@ -12,8 +12,8 @@ namespace moe {
 namespace {
 
 struct WsLayout {
-  size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, w1_deq, w2_deq, tok16,
-      route_partial, total;
+  size_t block_counts, topk_idx, topk_w, counts, offsets, perm, inv, x_perm, h, o_perm, xq, x_sf, hq, h_sf,
+      mx_prep, route_partial, total;
 };
 
 WsLayout ws_layout(const moe_dims_t& d) {
@@ -37,12 +37,14 @@ WsLayout ws_layout(const moe_dims_t& d) {
   L.o_perm = take(static_cast<size_t>(R) * d.D * 4);
   if (route_splits(d) > 1)  // K-split router: fp32 partial logits per split
     L.route_partial = take(static_cast<size_t>(route_splits(d)) * d.T * ((d.E + 15) / 16 * 16) * 4);
-  if (stream_fp4_applies(d)) {
-    // routed rows (x_perm, then h) in f16 for the weight-streaming MXFP4 kernels
-    L.tok16 = take(static_cast<size_t>(R) * (d.D > d.I ? d.D : d.I) * 2);
-  } else if (d.wfmt == MOE_W_MXFP4) {
-    L.w1_deq = take(static_cast<size_t>(d.E) * 2 * d.I * d.D * 2);
-    L.w2_deq = take(static_cast<size_t>(d.E) * d.D * d.I * 2);
+  if (d.wfmt == MOE_W_MXFP4) {
+    // block-scaled MMA operands: the routed rows and h as hi/lo E4M3 pairs
+    // plus their tile-blocked E8M0 scales (the expert weights are used as stored)
+    L.xq = take(static_cast<size_t>(R) * d.D * 2);
+    L.x_sf = take(mx_sf_bytes(d, d.D));
+    L.hq = take(static_cast<size_t>(R) * d.I * 2);
+    L.h_sf = take(mx_sf_bytes(d, d.I));
+    L.mx_prep = take(mx_prep_bytes(d));
   }
   L.total = off;
   return L;
@@ -89,19 +91,6 @@ bool use_pair(const moe_dims_t& d) { return static_cast<int64_t>(d.T) * d.k >= 2
   do {                                            \
     if (!(cond)) return MOE_ERR_INVALID_ARG;      \
   } while (0)
-
-// bf16 view of an expert weight: the tensor itself, or its expansion in ws.
-moe_status_t weight_bf16(const moe_dims_t& d, const moe_weight_t& w, int64_t N, int64_t K, void* ws, size_t deq_off,
-                         cudaStream_t s, const uint16_t** out) {
-  if (d.wfmt == MOE_W_BF16) {
-    *out = static_cast<const uint16_t*>(w.data);
-    return MOE_OK;
-  }
-  uint16_t* deq = at<uint16_t>(ws, deq_off);
-  MOE_TRY(cuda_status(launch_dequant_mxfp4(static_cast<const uint8_t*>(w.data), w.scales, d.E, N, K, deq, s)));
-  *out = deq;
-  return MOE_OK;
-}
 
 }  // namespace
 }  // namespace moe
@@ -166,11 +155,15 @@ moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offse
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(d);
-  if (stream_fp4_applies(d))
-    return launch_mlp1_fp4_stream(d, x_perm, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h,
-                                  at<uint16_t>(ws, L.tok16), status_word(ws), s);
-  const uint16_t* w1 = nullptr;
-  MOE_TRY(weight_bf16(d, W1, 2 * static_cast<int64_t>(d.I), d.D, ws, L.w1_deq, s, &w1));
+  if (d.wfmt == MOE_W_MXFP4) {
+    // the routed rows to hi/lo E4M3 + scales, then the block-scaled GEMM (h in bf16)
+    MOE_TRY(launch_mx_quant(d, x_perm, nullptr, d.D, offsets, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.x_sf),
+                            status_word(ws), s));
+    return launch_mlp1_mx(d, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.x_sf), offsets,
+                          static_cast<const uint8_t*>(W1.data), W1.scales, b1, h, nullptr, nullptr,
+                          at<uint8_t>(ws, L.mx_prep), status_word(ws), s);
+  }
+  const uint16_t* w1 = static_cast<const uint16_t*>(W1.data);
   if (use_pair(d)) return launch_mlp1_pair(d, x_perm, offsets, w1, b1, h, status_word(ws), s);
   return launch_mlp1(d, x_perm, offsets, w1, b1, h, status_word(ws), s);
 }
@@ -184,11 +177,14 @@ moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, cons
   MOE_TRY(check_ws(d, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(d);
-  if (stream_fp4_applies(d))
-    return launch_mlp2_fp4_stream(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
-                                  o_perm, at<uint16_t>(ws, L.tok16), status_word(ws), s);
-  const uint16_t* w2 = nullptr;
-  MOE_TRY(weight_bf16(d, W2, d.D, d.I, ws, L.w2_deq, s, &w2));
+  if (d.wfmt == MOE_W_MXFP4) {
+    MOE_TRY(launch_mx_quant(d, h, nullptr, d.I, offsets, at<uint8_t>(ws, L.hq), at<uint8_t>(ws, L.h_sf),
+                            status_word(ws), s));
+    return launch_mlp2_mx(d, at<uint8_t>(ws, L.hq), at<uint8_t>(ws, L.h_sf), perm, offsets, topk_w,
+                          static_cast<const uint8_t*>(W2.data), W2.scales, b2, o_perm, at<uint8_t>(ws, L.mx_prep),
+                          status_word(ws), s);
+  }
+  const uint16_t* w2 = static_cast<const uint16_t*>(W2.data);
   if (use_pair(d)) return launch_mlp2_pair(d, h, perm, offsets, topk_w, w2, b2, o_perm, status_word(ws), s);
   return launch_mlp2(d, h, perm, offsets, topk_w, w2, b2, o_perm, status_word(ws), s);
 }
@@ -202,21 +198,21 @@ moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* per
   const WsLayout L = ws_layout(d);
   uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
   uint16_t* h = at<uint16_t>(ws, L.h);
-  if (stream_fp4_applies(d)) {
-    // MXFP4 weight streaming: x_perm and h are internal here, so the gather
-    // writes the routed rows straight into the f16 form the kernels read and
-    // mlp1 writes h in mlp2's input form (the same values the stage-by-stage
-    // entry points produce with their conversion passes)
+  if (d.wfmt == MOE_W_MXFP4) {
+    // x_perm and h are internal here: the gather writes the routed rows
+    // straight into their hi/lo E4M3 form and mlp1 writes h in the same form
+    // (the same values the stage-by-stage entry points produce)
     MOE_REQUIRE(x && aligned32(x) && aligned32(b1) && aligned32(b2) && aligned32(o_perm));
     MOE_TRY(check_weight(d, W1));
     MOE_TRY(check_weight(d, W2));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint16_t* tok16 = at<uint16_t>(ws, L.tok16);
-    MOE_TRY(cuda_status(launch_gather(d, x, perm, tok16, status_word(ws), s, true)));
-    MOE_TRY(launch_mlp1_fp4_stream(d, tok16, offsets, static_cast<const uint8_t*>(W1.data), W1.scales, b1, h, tok16,
-                                   status_word(ws), s, true, true));
-    return launch_mlp2_fp4_stream(d, h, perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data), W2.scales, b2,
-                                  o_perm, tok16, status_word(ws), s, true);
+    uint8_t* xq = at<uint8_t>(ws, L.xq);
+    uint8_t* hq = at<uint8_t>(ws, L.hq);
+    MOE_TRY(launch_mx_quant(d, x, perm, d.D, offsets, xq, at<uint8_t>(ws, L.x_sf), status_word(ws), s));
+    MOE_TRY(launch_mlp1_mx(d, xq, at<uint8_t>(ws, L.x_sf), offsets, static_cast<const uint8_t*>(W1.data), W1.scales,
+                           b1, nullptr, hq, at<uint8_t>(ws, L.h_sf), at<uint8_t>(ws, L.mx_prep), status_word(ws), s));
+    return launch_mlp2_mx(d, hq, at<uint8_t>(ws, L.h_sf), perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data),
+                          W2.scales, b2, o_perm, at<uint8_t>(ws, L.mx_prep), status_word(ws), s);
   }
   MOE_TRY(moe_gather(d, x, perm, x_perm, ws, ws_bytes, stream));
   MOE_TRY(moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, ws_bytes, stream));

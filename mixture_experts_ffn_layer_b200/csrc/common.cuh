@@ -95,24 +95,24 @@ moe_status_t launch_mlp2_pair(const moe_dims_t& d, const uint16_t* h, const int3
                               const float* topk_w, const uint16_t* W2, const uint16_t* b2, float* o_perm,
                               int* status, cudaStream_t s);
 
-// MXFP4 weights with few routed rows per expert (stream_fp4.cu): the codes
-// are streamed from HBM once and decoded on chip into tcgen05 operands; no
-// expansion pass. Applies when the experts average at most 16 routed rows.
-bool stream_fp4_applies(const moe_dims_t& d);
-// in_f16: x_perm already holds the routed rows in f16 (no conversion pass);
-// h_f16: write h as f16(bf16(h) * 2^-8), the form mlp2's kernel reads.
-moe_status_t launch_mlp1_fp4_stream(const moe_dims_t& d, const uint16_t* x_perm, const int32_t* offsets,
-                                    const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                                    uint16_t* tok16, int* status, cudaStream_t s, bool in_f16 = false,
-                                    bool h_f16 = false);
-// in_f16: h already holds f16(bf16(h) * 2^-8) (mlp1 with h_f16).
-moe_status_t launch_mlp2_fp4_stream(const moe_dims_t& d, const uint16_t* h, const int32_t* perm,
-                                    const int32_t* offsets, const float* topk_w, const uint8_t* codes,
-                                    const uint8_t* scales, const uint16_t* b2, float* o_perm, uint16_t* tok16,
-                                    int* status, cudaStream_t s, bool in_f16 = false);
-
-// MXFP4 -> bf16 expansion of an (E, N, K) expert weight (mxfp4.cu).
-cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t E, int64_t N, int64_t K,
-                                 uint16_t* out, cudaStream_t s);
+// MXFP4 expert weights on block-scaled tcgen05 MMA (mx_gemm.cu). The
+// activations (routed rows, h) are quantised to hi/lo E4M3 pairs with E8M0
+// scales per 32 elements; the scales are stored tile-blocked, mx_sf_bytes
+// bytes for a reduction length K.
+size_t mx_sf_bytes(const moe_dims_t& d, int K);
+// Workspace each MX GEMM needs for its weights' per-stage scale atoms (and,
+// with a ragged K, the padded last codes of every weight row); one region
+// serves mlp1 and mlp2 in turn.
+size_t mx_prep_bytes(const moe_dims_t& d);
+// src rows (with perm: the gather x[perm[r] / k]) -> dst = hi (R, K) then lo (R, K), sf.
+moe_status_t launch_mx_quant(const moe_dims_t& d, const uint16_t* src, const int32_t* perm, int K,
+                             const int32_t* offsets, uint8_t* dst, uint8_t* sf, int* status, cudaStream_t s);
+// mlp1 from quantised rows; h in bf16 (h non-null) or quantised for mlp2 (hq, h_sf).
+moe_status_t launch_mlp1_mx(const moe_dims_t& d, const uint8_t* xq, const uint8_t* x_sf, const int32_t* offsets,
+                            const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
+                            uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s);
+moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_t* h_sf, const int32_t* perm,
+                            const int32_t* offsets, const float* topk_w, const uint8_t* codes, const uint8_t* scales,
+                            const uint16_t* b2, float* o_perm, uint8_t* prep, int* status, cudaStream_t s);
 
 }  // namespace moe

@@ -1,0 +1,751 @@
+// Grouped expert GEMMs with MXFP4 expert weights on block-scaled tcgen05 MMA.
+//
+// MXFP4 (GPT-OSS in Transformers blog, MXFP4 paragraph): E2M1 4-bit values
+// with one E8M0 scale per 32 consecutive elements of the reduction dim; the
+// torchtitan GPT-OSS guide ("grouped matrix multiplication") runs the expert
+// FFN as two grouped GEMMs over the expert segments of the routed rows.
+//
+// The sm_100a tensor cores multiply MX operands directly
+// (tcgen05.mma kind::mxf8f6f4.block_scale: per-32-element E8M0 scales for
+// both operands, read from tensor memory), but both operands must be MX
+// types. The weights stay E2M1 as stored; the bf16 activations (routed rows,
+// then h) are quantised to MX E4M3 as a PAIR of terms per element, hi + lo,
+// each with its own E8M0 scale per 32 elements:
+//   hi = e4m3(v / 2^(e-7)),  lo = e4m3((v - hi*2^(e-7)) / 2^(e_r-7)),
+// e and e_r the binary exponents of the block's largest |v| and largest
+// residual. hi keeps 4 significant bits, lo the next 4, so the pair carries
+// ~8 bits like bf16 itself (one E4M3 alone would leave errors of ~2^-5 per
+// element, too coarse for the layer's output). The two MMAs (hi, lo) per K
+// block accumulate into the same fp32 accumulator; every weight byte crosses
+// HBM and L2 at 4.25 bits per element and is never expanded.
+//
+// One persistent, warp-specialised kernel for mlp1 (+bias, SwiGLU) and mlp2
+// (+bias, gate weight); tiles are (expert, column tile, 128-row tile) over
+// the device-side expert offsets, as in the bf16 grouped GEMM:
+//   warp 0      producer, per 128-K stage: the tile's 128 activation rows as
+//               hi and lo E4M3 boxes (TMA, 128-byte swizzle) and their 1 KB of
+//               scale factors (bulk copy); the weight rows' E2M1 codes (TMA
+//               with the 16U4_ALIGN16B type, which unpacks every 8 bytes of
+//               codes into the 16-byte slot the MMA's E2M1 operand layout
+//               wants) and their 1 KB of scale factors (bulk copy);
+//   warp 1      MMA: tcgen05.cp of the stage's scale factors into tensor
+//               memory, then per 32-K block two block-scaled MMAs (hi, lo),
+//               M = 128 rows, N = the tile's weight rows; whole warp, one
+//               elected lane issuing;
+//   warps 2..5  epilogue: bias + SwiGLU into h (bf16, or straight into the
+//               quantised hi/lo form mlp2 reads), or bias * gate weight into
+//               the fp32 expert outputs.
+//
+// Scale factors reach tensor memory through tcgen05.cp, which reads 128 rows'
+// scales of 4 K blocks as a 32 x 16-byte shared-memory atom (row m's scale
+// of block kb at byte (m % 32) * 16 + (m / 32) * 4 + kb). Both operands'
+// scales are stored in that form in global memory, so a stage moves them
+// with one bulk copy each:
+//  - activations, tile-blocked: for m-tile g (the 128-row tiles of all
+//    experts, numbered expert by expert) and stage q, 1 KB at (g * nst + q) *
+//    1024 (hi atom, then lo atom), written by the quantiser / mlp1's epilogue;
+//  - weights, per (expert, column tile, stage): 1 KB (two atoms, rows 0..127
+//    and 128..255 of the tile), written from the (E, N, K/32) scales by a
+//    preparation pass before each GEMM (13 MB read at the 20B shape).
+// TMA's 4-bit type needs K to be a multiple of 128; for K % 128 = 64
+// (GPT-OSS: 2880) the same pass writes each weight row's last 64 codes
+// padded with zeros to a 128-element row, loaded by a second tensor map.
+//
+// Every mbarrier wait is bounded (1 s); on timeout the kernel records
+// MOE_ERR_TIMEOUT, stops issuing, waits for its in-flight copies and MMAs,
+// frees TMEM and returns.
+#include <cuda_fp16.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "sm100.cuh"
+#include "tma_host.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;                                   // token rows per tile = TMEM lanes
+constexpr int BKE = 128;                                  // K elements per stage (4 scale blocks)
+constexpr int kStages = 3;
+constexpr int kThreads = 192;                             // producer, MMA, 4 epilogue warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccStride = 256;                      // accumulators at columns 0 and 256
+// Two 16-column scale-factor regions, used by alternate stages: after
+// accumulator 0 (columns 240..255) and after accumulator 1 (496..511).
+constexpr uint32_t kSfCol0 = 240, kSfCol1 = 496;
+constexpr int kMaxN = 240;                                // MMA N (weight rows per tile) at most
+constexpr uint32_t kAOpBytes = BM * BKE;                  // one E4M3 operand box: 16 KB
+constexpr uint32_t kAStageBytes = 2 * kAOpBytes + 1024;   // hi, lo, their scale atoms
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr int kCtrlBytes = 256;
+
+struct MxParams {
+  GemmParams g;            // sizes, bias, perm / gate weights, output, status, activation
+  int nst;                 // 128-K stages
+  int kfull;               // K rounded down to a multiple of 128 (the rest comes from the tail rows)
+  const uint8_t* a_sf;     // activation scales, tile-blocked (nst stages)
+  const uint8_t* w_sf;     // weight scales: 1 KB per (expert, column tile, stage)
+  uint8_t* hq;             // mlp1, optional: h quantised, hi (R, I) then lo (R, I) E4M3
+  uint8_t* h_sf;           // and its scales, tile-blocked with h_nst stages
+  int h_nst;
+};
+
+// One stage: A hi, A lo, A scale atoms, the B operand (mma_n rows of 128
+// bytes), B scale atoms (two of 512 bytes), rounded up to 1 KB.
+__host__ __device__ constexpr uint32_t stage_bytes(int mma_n) {
+  return kAStageBytes + (static_cast<uint32_t>(mma_n) * 128 + 1024 + 1023) / 1024 * 1024;
+}
+
+__device__ __forceinline__ uint32_t sf_atom_off(int m, int kb) {
+  return static_cast<uint32_t>((m & 31) * 16 + (m >> 5) * 4 + kb);
+}
+
+// ---------------------------------------------------------------- E4M3 hi/lo quantisation
+// Two fp32 -> two E4M3 (round to nearest even, saturating), `a` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Two E4M3 (low byte first) -> their exact values.
+__device__ __forceinline__ float2 e4m3x2_value(uint32_t v) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(v)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+// 32 consecutive values of one row -> their hi and lo E4M3 codes (32 bytes
+// each, element i in byte i) and E8M0 scale bytes. A block whose largest |v|
+// is below 2^-119 is taken as zero (its terms are below 2^-119 * sum|w|); a
+// non-finite value makes the whole block NaN, which the MMA propagates.
+__device__ __forceinline__ void quant32(const float (&v)[32], uint32_t (&hi)[8], uint32_t (&lo)[8], uint32_t& sfh,
+                                        uint32_t& sfl) {
+  float amax = 0.f, chk = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    amax = fmaxf(amax, fabsf(v[i]));
+    chk += v[i] * 0.f;  // NaN if any value is inf or NaN
+  }
+  if (chk != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi[i] = lo[i] = 0x7f7f7f7fu;
+    sfh = sfl = 127;
+    return;
+  }
+  if (!(amax >= 0x1p-119f)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi[i] = lo[i] = 0u;
+    sfh = sfl = 127;
+    return;
+  }
+  // scale 2^(e-7) puts the block's largest value in [128, 256), inside E4M3's 448
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+  const float mul = __uint_as_float(static_cast<uint32_t>(127 + 7 - e) << 23);
+  const float back = __uint_as_float(static_cast<uint32_t>(127 + e - 7) << 23);
+  sfh = static_cast<uint32_t>(e + 120);
+  float r[32];
+  float rmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = e4m3x2(v[2 * i] * mul, v[2 * i + 1] * mul);
+    const float2 d = e4m3x2_value(q);
+    r[2 * i] = v[2 * i] - d.x * back;
+    r[2 * i + 1] = v[2 * i + 1] - d.y * back;
+    rmax = fmaxf(rmax, fmaxf(fabsf(r[2 * i]), fabsf(r[2 * i + 1])));
+    if (i & 1)
+      hi[i >> 1] |= q << 16;
+    else
+      hi[i >> 1] = q;
+  }
+  if (!(rmax >= 0x1p-119f)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lo[i] = 0u;
+    sfl = 127;
+    return;
+  }
+  const int er = static_cast<int>((__float_as_uint(rmax) >> 23) & 0xffu) - 127;
+  const float mul2 = __uint_as_float(static_cast<uint32_t>(127 + 7 - er) << 23);
+  sfl = static_cast<uint32_t>(er + 120);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = e4m3x2(r[2 * i] * mul2, r[2 * i + 1] * mul2);
+    if (i & 1)
+      lo[i >> 1] |= q << 16;
+    else
+      lo[i >> 1] = q;
+  }
+}
+
+// Expert segment table and m-tile prefix (numbering of the 128-row tiles of
+// all experts, expert by expert) from the offsets, into shared memory, by one
+// warp; returns false (and records the status) for offsets out of order or
+// range. mpre has E+1 entries.
+__device__ bool load_segments(const int32_t* offsets, int E, int64_t R, int* seg, int* mpre, int* status) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  for (int e = lane; e <= E; e += 32) {
+    const int o = offsets[e];
+    seg[e] = o;
+    if (o < 0 || o > R || (e == 0 && o != 0)) bad = true;
+  }
+  __syncwarp();
+  const int per = (E + 31) / 32;
+  const int e0 = lane * per;
+  int local = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int cnt = seg[e + 1] - seg[e];
+    if (cnt < 0) bad = true;
+    local += cnt > 0 ? (cnt + BM - 1) / BM : 0;
+  }
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  int run = incl - local;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    mpre[e] = run;
+    const int cnt = seg[e + 1] - seg[e];
+    run += cnt > 0 ? (cnt + BM - 1) / BM : 0;
+  }
+  if (lane == 31) mpre[E] = incl;
+  __syncwarp();
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad && lane == 0) record_status(status, MOE_ERR_DEVICE_BOUNDS);
+  return !bad;
+}
+
+// ---------------------------------------------------------------- quantiser kernel
+// Rows of `src` (bf16; with `perm`, row r is x[perm[r] / k], the gather of
+// the routed rows) -> hi (R, K) and lo (R, K) E4M3 at dst and dst + R*K, and
+// their scales in the tile-blocked layout. One thread per 32-element block.
+__global__ void __launch_bounds__(256) mx_quant_kernel(const uint16_t* __restrict__ src, const int32_t* __restrict__ perm,
+                                                       int k, int64_t R, int K, const int32_t* __restrict__ offsets,
+                                                       int E, int nst, uint8_t* __restrict__ dst,
+                                                       uint8_t* __restrict__ sf, int* status) {
+  __shared__ int seg[257], mpre[257];
+  __shared__ int ok_s;
+  if (threadIdx.x < 32) {
+    const bool ok = load_segments(offsets, E, R, seg, mpre, status);
+    if (threadIdx.x == 0) ok_s = ok;
+  }
+  __syncthreads();
+  if (!ok_s) return;
+  const int nb = K / 32;
+  const int64_t total = R * nb;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nb;
+    const int b = static_cast<int>(i - r * nb);
+    int64_t srow = r;
+    if (perm) {
+      const int32_t a = perm[r];
+      if (a < 0 || a >= R) {
+        if (b == 0) record_status(status, MOE_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      srow = a / k;
+    }
+    uint32_t w[16];
+    ld_global_v8u(src + srow * K + 32 * b, *reinterpret_cast<uint32_t(*)[8]>(w));
+    ld_global_v8u(src + srow * K + 32 * b + 16, *reinterpret_cast<uint32_t(*)[8]>(w + 8));
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+    uint32_t hi[8], lo[8], sfh, sfl;
+    quant32(v, hi, lo, sfh, sfl);
+    st_global_v8u(dst + r * K + 32 * b, hi);
+    st_global_v8u(dst + R * K + r * K + 32 * b, lo);
+    // the row's expert (last e with seg[e] <= r among non-empty ones) and tile
+    int lo_e = 0, hi_e = E - 1;
+    while (lo_e < hi_e) {
+      const int mid = (lo_e + hi_e + 1) >> 1;
+      if (seg[mid] <= r)
+        lo_e = mid;
+      else
+        hi_e = mid - 1;
+    }
+    const int local = static_cast<int>(r - seg[lo_e]);
+    const int64_t g = mpre[lo_e] + local / BM;
+    uint8_t* atom = sf + (g * nst + b / 4) * 1024;
+    const uint32_t o = sf_atom_off(local % BM, b % 4);
+    atom[o] = static_cast<uint8_t>(sfh);
+    atom[512 + o] = static_cast<uint8_t>(sfl);
+  }
+}
+
+// ---------------------------------------------------------------- weight preparation
+// Weight scales -> per (expert, column tile, stage) 1 KB atoms; with K % 128
+// = 64, each weight row's last 64 codes padded to a 128-element row. One
+// thread per 4 scale bytes (a row of a tile's stage) or per 16 bytes of tail.
+__global__ void __launch_bounds__(256) mx_prep_weights_kernel(const uint8_t* __restrict__ codes,
+                                                              const uint8_t* __restrict__ scales, int E, int b_rows,
+                                                              int K, int n_out, int n_tile, int mma_n, int NT,
+                                                              int nst, int swiglu, uint8_t* __restrict__ w_sf,
+                                                              uint8_t* __restrict__ tail) {
+  const int nsc = K / 32, half_k = K / 2, kfull = K / BKE * BKE;
+  const int64_t n_atoms = static_cast<int64_t>(E) * NT * nst * mma_n;
+  const int64_t n_tail = kfull < K ? static_cast<int64_t>(E) * b_rows * 4 : 0;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_atoms + n_tail;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (i < n_atoms) {
+      const int j = static_cast<int>(i % mma_n);
+      const int64_t tq = i / mma_n;  // (e * NT + nt) * nst + q
+      const int q = static_cast<int>(tq % nst);
+      const int64_t ent = tq / nst;
+      const int nt = static_cast<int>(ent % NT), e = static_cast<int>(ent / NT);
+      const int64_t row = static_cast<int64_t>(e) * b_rows +
+                          (swiglu ? (j < n_tile ? nt * n_tile + j : n_out + nt * n_tile + (j - n_tile))
+                                  : nt * n_tile + j);
+      const uint16_t* s2 = reinterpret_cast<const uint16_t*>(scales + row * nsc + q * 4);
+      const uint32_t lo16 = __ldg(s2);
+      const uint32_t hi16 = q * 4 + 2 < nsc ? static_cast<uint32_t>(__ldg(s2 + 1)) : 0x7f7fu;
+      *reinterpret_cast<uint32_t*>(w_sf + tq * 1024 + (j >> 7) * 512 + sf_atom_off(j & 127, 0)) = lo16 | (hi16 << 16);
+    } else {
+      const int64_t t = i - n_atoms;
+      const int64_t row = t >> 2;
+      const int piece = static_cast<int>(t & 3);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (piece < 2) v = __ldg(reinterpret_cast<const uint4*>(codes + row * half_k + kfull / 2 + piece * 16));
+      *reinterpret_cast<uint4*>(tail + row * 64 + piece * 16) = v;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- the block-scaled grouped GEMM
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmAhi, const __grid_constant__ CUtensorMap tmAlo,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBtail,
+                   const MxParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const GemmParams& gp = p.g;
+  const uint32_t sst = stage_bytes(gp.mma_n);
+  constexpr uint32_t kBOff = kAStageBytes;                                 // B operand within a stage
+  const uint32_t sfb_off = kBOff + static_cast<uint32_t>(gp.mma_n) * 128;  // B scale atoms within a stage
+  uint8_t* ring = smem;
+  uint8_t* ctrl = ring + kStages * sst;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
+  constexpr int kBars = 2 * kStages + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* seg = reinterpret_cast<int*>(ctrl + kCtrlBytes);
+  int* mpre = seg + (gp.E + 1);
+  int* tpre = mpre + (gp.E + 1);
+
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (2 * kStages + 4);
+
+  // ---- prologue: segments, tile prefixes, barriers, TMEM
+  if (warp == 0) {
+    const bool ok = load_segments(gp.offsets, gp.E, gp.R, seg, mpre, gp.status);
+    for (int e = lane; e <= gp.E; e += 32) tpre[e] = mpre[e] * gp.NT;
+    __syncwarp();
+    if (lane == 0) {
+      *abort_flag = 0;
+      *total_s = ok ? tpre[gp.E] : 0;
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(full_bar(s), 1);
+        mbar_init(empty_bar(s), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(tfull(b), 1);
+        mbar_init(tempty(b), 4);
+      }
+      mbar_init(done_bar, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmAhi);
+      tma_prefetch_desc(&tmAlo);
+      if (p.kfull > 0) tma_prefetch_desc(&tmB);
+      if (p.kfull < gp.K) tma_prefetch_desc(&tmBtail);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // All 512 columns are allocated, so the allocation starts at lane 0, column
+  // 0; TMEM is addressed from that constant (warp-uniform operands).
+  const uint32_t tmem_got = *tmem_slot;
+  constexpr uint32_t tmem_base = 0;
+  if (tmem_got != tmem_base && threadIdx.x == 0) record_status(gp.status, MOE_ERR_CUDA);
+  const int total = tmem_got == tmem_base ? *total_s : 0;
+  const int nst = p.nst;
+  const int nfull = p.kfull / BKE;  // stages whose codes come from the weights; the last, if ragged, from the tail rows
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      const uint32_t stage_tx = kAStageBytes + static_cast<uint32_t>(gp.mma_n) * (BKE / 2) + 1024;
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+        int e, nt, mt;
+        decode_tile(tile, tpre, seg, gp.E, BM, e, nt, mt);
+        const int row0 = seg[e] + mt * BM;
+        const int64_t g = mpre[e] + mt;
+        const int brow = e * gp.b_rows + nt * gp.n_tile;
+        const uint8_t* wsf = p.w_sf + (static_cast<int64_t>(e) * gp.NT + nt) * nst * 1024;
+        for (int q = 0; q < nst; ++q) {
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
+            failed = true;
+            break;
+          }
+          const uint32_t st = smem_u32(ring + s * sst);
+          mbar_arrive_expect_tx(full_bar(s), stage_tx);
+          tma_load_2d(st, &tmAhi, full_bar(s), q * BKE, row0);
+          tma_load_2d(st + kAOpBytes, &tmAlo, full_bar(s), q * BKE, row0);
+          bulk_load(st + 2 * kAOpBytes, p.a_sf + (g * nst + q) * 1024, 1024, full_bar(s));
+          const CUtensorMap* tb = q < nfull ? &tmB : &tmBtail;
+          const int bx = q < nfull ? q * BKE : 0;
+          tma_load_2d(st + kBOff, tb, full_bar(s), bx, brow);
+          if (kSwiGLU) tma_load_2d(st + kBOff + gp.n_tile * 128, tb, full_bar(s), bx, brow + gp.n_out);
+          bulk_load(st + sfb_off, wsf + q * 1024, 1024, full_bar(s));
+          ++issued;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (failed) {
+        record_status(gp.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        const int n = issued < kStages ? issued : kStages;  // copies still in flight
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = kStages - 1;
+            ph ^= 1u;
+          }
+          mbar_wait_bounded(full_bar(s), ph, nullptr, kWaitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs the loop and one elected lane issues each tcgen05
+    // instruction, so every operand is warp-uniform.
+    const uint32_t idesc = idesc_mx(0 /* E4M3 */, 5 /* E2M1 */, gp.mma_n);
+    int s = 0, acc = 0, sfr = 0;
+    uint32_t ph = 0, pacc = 0;
+    bool failed = false;
+    for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tempty(acc), pacc ^ 1u, abort_flag, kWaitNs))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kAccStride;
+      for (int q = 0; q < nst; ++q) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(ring + s * sst);
+        const uint32_t b = st + kBOff;
+        const uint32_t tsf = tmem_base + (sfr ? kSfCol1 : kSfCol0);
+        sfr ^= 1;
+        tc_cp_sf_elect(tsf + 0, desc_noswizzle(st + 2 * kAOpBytes, 128));
+        tc_cp_sf_elect(tsf + 4, desc_noswizzle(st + 2 * kAOpBytes + 512, 128));
+        tc_cp_sf_elect(tsf + 8, desc_noswizzle(st + sfb_off, 128));
+        if (gp.mma_n > 128) tc_cp_sf_elect(tsf + 12, desc_noswizzle(st + sfb_off + 512, 128));
+        const int kleft = gp.K - q * BKE;
+        const int nkb = kleft >= BKE ? 4 : kleft / 32;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint64_t bd = desc_kmajor_sw128(b + kb * 32);
+          mma_mx_elect(d_tmem, desc_kmajor_sw128(st + kb * 32), bd, idesc, kb, tsf + 0, tsf + 8,
+                       (q | kb) != 0 ? 1u : 0u);
+          mma_mx_elect(d_tmem, desc_kmajor_sw128(st + kAOpBytes + kb * 32), bd, idesc, kb, tsf + 4, tsf + 8, 1u);
+        }
+        tc_commit_elect(empty_bar(s));
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (failed) break;
+      tc_commit_elect(tfull(acc));
+      if (++acc == 2) {
+        acc = 0;
+        pacc ^= 1u;
+      }
+    }
+    if (failed && lane == 0) {
+      record_status(gp.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    tc_commit_elect(done_bar);
+    mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    const int m = qd * 32 + lane;
+    int acc = 0;
+    uint32_t pacc = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, nt, mt;
+      decode_tile(tile, tpre, seg, gp.E, BM, e, nt, mt);
+      const bool ok = mbar_wait_bounded(tfull(acc), pacc, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          record_status(gp.status, MOE_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(seg[e]) + mt * BM + m;
+      const bool valid = row < seg[e + 1];
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kAccStride;
+      if (kSwiGLU && p.hq != nullptr) {
+        // bias + activation, h rounded to bf16, then straight into mlp2's
+        // operand form: hi/lo E4M3 + scales (the quantiser's arithmetic)
+        const uint16_t* bg = gp.bias + static_cast<int64_t>(e) * gp.b_rows + nt * gp.n_tile;
+        const uint16_t* bu = bg + gp.n_out;
+        const int64_t g = mpre[e] + mt;
+        for (int c0 = 0; c0 < gp.n_tile; c0 += 32) {
+          float v[32];
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time keeps the registers in check
+            uint32_t ga[16], ua[16];
+            tmem_ld_x8(tbase + c0 + 16 * hf, ga);
+            tmem_ld_x8(tbase + c0 + 16 * hf + 8, ga + 8);
+            tmem_ld_x8(tbase + gp.n_tile + c0 + 16 * hf, ua);
+            tmem_ld_x8(tbase + gp.n_tile + c0 + 16 * hf + 8, ua + 8);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              float gb[8], ub[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(bg + c0 + 16 * hf + 8 * j)), gb);
+              unpack8(__ldg(reinterpret_cast<const uint4*>(bu + c0 + 16 * hf + 8 * j)), ub);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float hv = glu_act(__uint_as_float(ga[8 * j + i]) + gb[i],
+                                         __uint_as_float(ua[8 * j + i]) + ub[i], gp.act);
+                v[16 * hf + 8 * j + i] = bf16_bits_to_float(float_to_bf16_bits(hv));
+              }
+            }
+          }
+          if (valid) {
+            uint32_t hi[8], lo[8], sfh, sfl;
+            quant32(v, hi, lo, sfh, sfl);
+            const int col = nt * gp.n_tile + c0;
+            st_global_v8u(p.hq + row * gp.n_out + col, hi);
+            st_global_v8u(p.hq + gp.R * gp.n_out + row * gp.n_out + col, lo);
+            uint8_t* atom = p.h_sf + (g * p.h_nst + col / BKE) * 1024;
+            const uint32_t o = sf_atom_off(m, (col % BKE) / 32);
+            atom[o] = static_cast<uint8_t>(sfh);
+            atom[512 + o] = static_cast<uint8_t>(sfl);
+          }
+        }
+      } else {
+        epilogue_tile<kSwiGLU>(gp, tbase, e, nt, row, valid);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(acc));
+      if (++acc == 2) {
+        acc = 0;
+        pacc ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_got, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+// (rows, inner) bytes, loaded as 128 x 128-byte boxes with the 128-byte
+// swizzle (the K-major E4M3 operand layout).
+bool make_tmap_e4m3(CUtensorMap* map, const uint8_t* base, uint64_t inner, uint64_t rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), static_cast<cuuint32_t>(BM)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E2M1 codes of `rows` rows of row_bytes bytes: the first kfull elements of
+// each row (kfull a multiple of 128) as 128-element x box_rows boxes,
+// unpacked by TMA into the MMA's E2M1 operand layout (every 8 bytes of codes
+// padded to 16) with the 128-byte swizzle. The base must be 32-byte aligned
+// and row_bytes a multiple of 32.
+bool make_tmap_e2m1(CUtensorMap* map, const uint8_t* codes, uint64_t kfull, uint64_t row_bytes, uint64_t rows,
+                    uint32_t box_rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {kfull, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t smem_bytes(int mma_n, int E) {
+  return 1024 + static_cast<size_t>(kStages) * stage_bytes(mma_n) + kCtrlBytes +
+         3 * static_cast<size_t>(E + 1) * sizeof(int);
+}
+
+int pick_tile(int n, int max_tile, int step) {
+  for (int t = max_tile; t >= step; t -= step)
+    if (n % t == 0) return t;
+  return 0;
+}
+
+// Tile sizes of the two GEMMs: mlp1 h columns per tile a multiple of 32
+// (whole scale blocks of mlp2's K), gate and up halves stacked in one MMA of
+// N = 2 * n_tile <= 240; mlp2 N = n_tile <= 240.
+int mlp1_ntile(const moe_dims_t& d) { return pick_tile(d.I, kMaxN / 2 / 32 * 32, 32); }
+int mlp2_ntile(const moe_dims_t& d) { return pick_tile(d.D, kMaxN, 16); }
+
+size_t w_sf_bytes(int E, int NT, int K) { return static_cast<size_t>(E) * NT * ((K + BKE - 1) / BKE) * 1024; }
+size_t w_tail_bytes(int E, int b_rows, int K) { return K % BKE ? static_cast<size_t>(E) * b_rows * 64 : 0; }
+
+template <bool kSwiGLU>
+moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8_t* scales, uint8_t* prep,
+                            MxParams p, cudaStream_t s) {
+  const GemmParams& g = p.g;
+  // weight scales into per-stage atoms (and the ragged-K tail rows) in prep
+  uint8_t* w_sf = prep;
+  uint8_t* tail = prep + align_up(w_sf_bytes(g.E, g.NT, g.K), 256);
+  {
+    const int64_t n = static_cast<int64_t>(g.E) * g.NT * p.nst * g.mma_n +
+                      (g.K % BKE ? static_cast<int64_t>(g.E) * g.b_rows * 4 : 0);
+    const int64_t blocks = (n + 255) / 256;
+    const int grid = static_cast<int>(blocks < 8 * num_sms() ? blocks : 8 * num_sms());
+    mx_prep_weights_kernel<<<grid, 256, 0, s>>>(codes, scales, g.E, g.b_rows, g.K, g.n_out, g.n_tile, g.mma_n, g.NT,
+                                                p.nst, kSwiGLU ? 1 : 0, w_sf, tail);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  p.w_sf = w_sf;
+  p.kfull = g.K / BKE * BKE;
+  CUtensorMap thi, tlo, tb, tt;
+  memset(&tb, 0, sizeof(tb));
+  memset(&tt, 0, sizeof(tt));
+  if (!make_tmap_e4m3(&thi, aq, g.K, g.R) || !make_tmap_e4m3(&tlo, aq + g.R * g.K, g.K, g.R)) return MOE_ERR_CUDA;
+  const uint64_t wrows = static_cast<uint64_t>(g.E) * g.b_rows;
+  const uint32_t box_rows = static_cast<uint32_t>(kSwiGLU ? g.n_tile : g.mma_n);
+  if (p.kfull > 0 && !make_tmap_e2m1(&tb, codes, p.kfull, g.K / 2, wrows, box_rows)) return MOE_ERR_CUDA;
+  if (p.kfull < g.K && !make_tmap_e2m1(&tt, tail, BKE, 64, wrows, box_rows)) return MOE_ERR_CUDA;
+  const size_t smem = smem_bytes(g.mma_n, g.E);
+  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(mx_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int64_t max_tiles = ((g.R + BM - 1) / BM + g.E) * static_cast<int64_t>(g.NT);
+  const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
+  mx_gemm_kernel<kSwiGLU><<<grid, kThreads, smem, s>>>(thi, tlo, tb, tt, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t mx_sf_bytes(const moe_dims_t& d, int K) {
+  const int64_t R = static_cast<int64_t>(d.T) * d.k;
+  return static_cast<size_t>((R + BM - 1) / BM + d.E) * ((K + BKE - 1) / BKE) * 1024;
+}
+
+size_t mx_prep_bytes(const moe_dims_t& d) {
+  const int n1 = mlp1_ntile(d), n2 = mlp2_ntile(d);
+  if (n1 == 0 || n2 == 0) return 0;
+  const size_t p1 = align_up(w_sf_bytes(d.E, d.I / n1, d.D), 256) + w_tail_bytes(d.E, 2 * d.I, d.D);
+  const size_t p2 = align_up(w_sf_bytes(d.E, d.D / n2, d.I), 256) + w_tail_bytes(d.E, d.D, d.I);
+  return align_up(p1 > p2 ? p1 : p2, 256);
+}
+
+moe_status_t launch_mx_quant(const moe_dims_t& d, const uint16_t* src, const int32_t* perm, int K,
+                             const int32_t* offsets, uint8_t* dst, uint8_t* sf, int* status, cudaStream_t s) {
+  const int64_t R = static_cast<int64_t>(d.T) * d.k;
+  const int64_t total = R * (K / 32);
+  const int64_t blocks = (total + 255) / 256;
+  const int grid = static_cast<int>(blocks < 8 * num_sms() ? blocks : 8 * num_sms());
+  mx_quant_kernel<<<grid, 256, 0, s>>>(src, perm, d.k, R, K, offsets, d.E, (K + BKE - 1) / BKE, dst, sf, status);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t launch_mlp1_mx(const moe_dims_t& d, const uint8_t* xq, const uint8_t* x_sf, const int32_t* offsets,
+                            const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
+                            uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s) {
+  const int nh = mlp1_ntile(d);
+  if (nh == 0) return MOE_ERR_UNSUPPORTED;
+  MxParams p{};
+  GemmParams& g = p.g;
+  g.E = d.E;
+  g.K = d.D;
+  g.n_out = d.I;
+  g.n_tile = nh;
+  g.mma_n = 2 * nh;
+  g.NT = d.I / nh;
+  g.b_rows = 2 * d.I;
+  g.R = static_cast<int64_t>(d.T) * d.k;
+  g.offsets = offsets;
+  g.bias = b1;
+  g.act = act_of(d);
+  g.out = h;
+  g.status = status;
+  p.nst = (d.D + BKE - 1) / BKE;
+  p.a_sf = x_sf;
+  p.hq = hq;
+  p.h_sf = h_sf;
+  p.h_nst = (d.I + BKE - 1) / BKE;
+  return launch_mx_gemm<true>(xq, codes, scales, prep, p, s);
+}
+
+moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_t* h_sf, const int32_t* perm,
+                            const int32_t* offsets, const float* topk_w, const uint8_t* codes, const uint8_t* scales,
+                            const uint16_t* b2, float* o_perm, uint8_t* prep, int* status, cudaStream_t s) {
+  const int nt = mlp2_ntile(d);
+  if (nt == 0) return MOE_ERR_UNSUPPORTED;
+  MxParams p{};
+  GemmParams& g = p.g;
+  g.E = d.E;
+  g.K = d.I;
+  g.n_out = d.D;
+  g.n_tile = nt;
+  g.mma_n = nt;
+  g.NT = d.D / nt;
+  g.b_rows = d.D;
+  g.R = static_cast<int64_t>(d.T) * d.k;
+  g.offsets = offsets;
+  g.bias = b2;
+  g.perm = perm;
+  g.topk_w = topk_w;
+  g.out = o_perm;
+  g.status = status;
+  p.nst = (d.I + BKE - 1) / BKE;
+  p.a_sf = h_sf;
+  return launch_mx_gemm<false>(hq, codes, scales, prep, p, s);
+}
+
+}  // namespace moe

@@ -257,6 +257,97 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 
+// ---------------------------------------------------------------- block-scaled MMA (MX formats)
+// Shared-memory descriptor of a tile without swizzle: 8-row core matrices
+// of 16-byte rows, consecutive core matrices `sbo` bytes apart (the source
+// layout of tcgen05.cp for scale factors).
+__device__ __forceinline__ uint64_t desc_noswizzle(uint32_t smem_addr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy 32 rows x 16 bytes of shared memory into 4 consecutive TMEM columns of
+// lanes 0..31, replicated to the other three lane quarters. With the scale
+// factors of 128 matrix rows laid out as 32 x 16 bytes (row m at byte
+// (m % 32) * 16 + (m / 32) * 4, one byte per 32-element K block), row m's
+// scale for K block kb lands in column m / 32, byte kb -- the layout the
+// block-scaled MMA reads.
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E8M0 block scales, M = 128,
+// K-major A and B, D fp32; a_fmt / b_fmt: 0 = E4M3, 5 = E2M1. The scale
+// factor byte used for both operands (K block within the 4-block TMEM word)
+// is added by mma_mx.
+__host__ __device__ constexpr uint32_t idesc_mx(int a_fmt, int b_fmt, int N) {
+  return (static_cast<uint32_t>(a_fmt) << 7) | (static_cast<uint32_t>(b_fmt) << 10) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// D[tmem] (+)= (A * sfA) * (B * sfB)^T over K = 32, A and B from shared
+// memory, the scale factors of K block kb (0..3) from TMEM words at sfa / sfb.
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, int kb,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  const uint32_t id = idesc | (static_cast<uint32_t>(kb) << 4) | (static_cast<uint32_t>(kb) << 29);
+  const uint32_t ta = sfa | (static_cast<uint32_t>(kb) << 30), tb = sfb | (static_cast<uint32_t>(kb) << 30);
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate), "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// The same two, executed by a whole warp with one lane elected to issue (the
+// operands then stay warp-uniform, which keeps the issue short).
+__device__ __forceinline__ void tc_cp_sf_elect(uint32_t taddr, uint64_t src_desc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(src_desc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mx_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, int kb,
+                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  const uint32_t id = idesc | (static_cast<uint32_t>(kb) << 4) | (static_cast<uint32_t>(kb) << 29);
+  const uint32_t ta = sfa | (static_cast<uint32_t>(kb) << 30), tb = sfb | (static_cast<uint32_t>(kb) << 30);
+  asm volatile(
+      "{\n\t.reg .pred e, q;\n\t.reg .b32 r;\n\t"
+      "setp.ne.b32 q, %4, 0;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], q;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate), "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns per thread.
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Plain shared-memory stores at a shared::cta address.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // ---------------------------------------------------------------- 2-CTA pairs (cluster of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -53,8 +53,9 @@ def test_check_dims_supported_set():
 
 def test_workspace_bytes_cover_the_decode_paths():
     # 64 tokens at the 20B shape: the router splits K over 45 CTAs (fp32
-    # partial logits, splits * T * E), and MXFP4 weights take the
-    # weight-streaming path (routed rows in f16) instead of expanding them
+    # partial logits, splits * T * E); MXFP4 weights add the block-scaled
+    # GEMMs' operands -- routed rows and h as hi/lo E4M3 pairs and their
+    # scales -- and never an expanded copy of the weights
     T, D, E, k, I = 64, 2880, 32, 4, 2880
     R = T * k
     base = R * D * (2 + 4) + R * I * 2 + R * 4 * 4
@@ -62,8 +63,13 @@ def test_workspace_bytes_cover_the_decode_paths():
     n = moe.workspace_bytes(moe.dims(T, D, E, k, I))
     assert base + splits * T * E * 4 <= n <= base + splits * T * E * 4 + 1024 * 1024
     nq = moe.workspace_bytes(moe.dims(T, D, E, k, I, wfmt=moe.MOE_W_MXFP4))
-    assert nq - n >= R * max(D, I) * 2  # routed rows in f16
-    assert nq - n < 2 * 2880 * 2880  # no expanded weights
+    mtiles = -(-R // 128) + E
+    sf = mtiles * -(-D // 128) * 1024 + mtiles * -(-I // 128) * 1024
+    # the weights' scales as per-stage atoms (E x 30 column tiles x 23 stages
+    # x 1 KB for mlp1) and the padded last 64 codes of every mlp1 weight row
+    prep = E * (I // 96) * -(-D // 128) * 1024 + E * 2 * I * 64
+    assert R * (D + I) * 2 + sf + prep <= nq - n <= R * (D + I) * 2 + sf + prep + 8192
+    assert nq - n < 64 * 1024 * 1024  # no expanded weights (1.59 GB at this shape)
 
 
 def test_workspace_bytes_covers_intermediates():
@@ -73,7 +79,8 @@ def test_workspace_bytes_covers_intermediates():
     need = R * 2880 * (2 + 2 + 4) + R * 4 * 4  # x_perm, h (bf16), o_perm (fp32) + idx, w, perm, inv
     assert need <= n <= need + 4 * 1024 * 1024
     dq = moe.dims(8192, 2880, 32, 4, 2880, wfmt=moe.MOE_W_MXFP4)
-    assert moe.workspace_bytes(dq) - n >= 32 * 3 * 2880 * 2880 * 2  # dequantized W1 and W2
+    extra = moe.workspace_bytes(dq) - n
+    assert R * 2880 * 4 <= extra <= R * 2880 * 4 + 64 * 1024 * 1024  # hi/lo operands + scales, no weight copies
     with pytest.raises(moe.MoeError):
         moe.workspace_bytes(moe.dims(8, 64, 4, 5, 64))
 

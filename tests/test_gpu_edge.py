@@ -55,17 +55,17 @@ def test_shapes(T, D, E, k, I):
     (96, 256, 24, 1, 192),  # non-power-of-two E
     (100, 128, 256, 8, 128),  # largest E and k: ~3 rows per expert, some experts empty
 ])
-def test_mxfp4_weight_streaming_shapes(T, D, E, k, I):
-    # at most 16 routed rows per expert on average: the MXFP4 weight-streaming kernels
+def test_mxfp4_small_batch_shapes(T, D, E, k, I):
+    # a few routed rows per expert (decode-like): most of each 128-row tile is padding
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + 7 * E, device="cuda", wfmt="mxfp4",
                                 reject=oracle.gap_reject())
     _check_full(inp, TOL_MXFP4)
 
 
-def test_mxfp4_hot_expert_several_passes():
-    # one expert takes most tokens: its rows span several 32-row passes, the
+def test_mxfp4_hot_expert_several_tiles():
+    # one expert takes most tokens: its rows span several 128-row tiles, the
     # last one ragged, while the other experts keep a few rows
-    T, D, E, k, I = 120, 128, 16, 2, 128
+    T, D, E, k, I = 400, 128, 16, 2, 128
     base = synthetic.make_custom(T, D, E, k, I, seed=11, wfmt="mxfp4")
     br = torch.zeros(E)
     br[5] = 6.0
@@ -75,14 +75,14 @@ def test_mxfp4_hot_expert_several_passes():
     shape = synthetic.LayerShape("custom", x.shape[0], D, E, k, I, wfmt="mxfp4")
     inp = dataclasses.replace(base, shape=shape, x=x, br=br).to("cuda")
     run = _check_full(inp, TOL_MXFP4)
-    assert int(run.counts.max()) > 64
+    assert int(run.counts.max()) > 256
 
 
 @pytest.mark.parametrize("T,D,E,k,I,wfmt", [
     (512, 256, 8, 2, 512, "bf16"),   # single-SM tcgen05 GEMM tiles
     (4200, 128, 4, 2, 192, "bf16"),  # SM-pair GEMM tiles
-    (40, 192, 8, 2, 320, "mxfp4"),   # MXFP4 weight-streaming kernels
-    (600, 128, 4, 2, 128, "mxfp4"),  # MXFP4 expanded to bf16, then the GEMM
+    (40, 192, 8, 2, 320, "mxfp4"),   # MXFP4, block-scaled MMA, a few rows per expert
+    (600, 128, 4, 2, 128, "mxfp4"),  # MXFP4, block-scaled MMA, several tiles per expert
 ])
 def test_gptoss_activation(T, D, E, k, I, wfmt):
     # the GPT-OSS SwiGLU variant in every mlp1 epilogue; a small limit so that
@@ -93,13 +93,15 @@ def test_gptoss_activation(T, D, E, k, I, wfmt):
 
 
 @pytest.mark.parametrize("T,D,E,k,I", [
-    (600, 128, 4, 2, 128),   # prefill-sized: weights expanded to bf16 in the workspace
+    (600, 128, 4, 2, 128),
     (1024, 256, 8, 4, 192),
-    (40, 192, 8, 2, 320),    # decode-sized: the one-call path feeds the weight-streaming
-    (64, 2880, 32, 4, 2880),  # kernels f16 rows from the gather and h from mlp1 directly
+    (40, 192, 8, 2, 320),
+    (64, 2880, 32, 4, 2880),
 ])
 def test_forward_mxfp4_matches_stages(T, D, E, k, I):
-    # the one-call MXFP4 path is bitwise the staged path, call after call
+    # the one-call MXFP4 path (the gather writes the hi/lo E4M3 operands, mlp1
+    # writes h in that form) is bitwise the staged path (bf16 x_perm and h,
+    # each quantised by its own pass), call after call
     inp = synthetic.make_custom(T, D, E, k, I, seed=T + E, device="cuda", wfmt="mxfp4", reject=oracle.gap_reject())
     run = run_stages(inp)
     assert run.status == 0
@@ -107,6 +109,53 @@ def test_forward_mxfp4_matches_stages(T, D, E, k, I):
     y2 = run_forward(inp)
     assert torch.equal(y1.view(torch.int16), run.y.view(torch.int16))
     assert torch.equal(y2.view(torch.int16), y1.view(torch.int16))
+
+
+@pytest.mark.parametrize("T", [40, 700])
+def test_mxfp4_wide_weight_scales(T):
+    # mlp2 weight rows whose E8M0 scales sit anywhere in a 60-binade range:
+    # every block of output row dd (all experts) is offset by the same o_dd in
+    # [-40, 20] binades (the synthetic workloads span 9 binades), and b2 = 0, so
+    # output column dd scales with 2^o_dd. Each column must match the oracle
+    # relative to its own magnitude: no block is flushed or rescaled against
+    # the other rows' or blocks' scales.
+    D, E, k, I = 256, 8, 2, 192
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + 1, wfmt="mxfp4", reject=oracle.gap_reject())
+    g = torch.Generator().manual_seed(T)
+    off = torch.randint(-40, 21, (1, D, 1), generator=g)
+    inp.W2_scales = (inp.W2_scales.long() + off).to(torch.uint8)
+    inp.b2 = torch.zeros_like(inp.b2)
+    inp = inp.to("cuda")
+    run = run_stages(inp)
+    assert run.status == 0
+    _, idx_ref, w_ref = oracle.route(inp.x, inp.Wr, inp.br, k)
+    assert torch.equal(run.topk_idx.cpu(), idx_ref)
+    _, y_ref = oracle.ffn_tokens(inp.x, idx_ref, w_ref, inp.W1, inp.b1, inp.W2, inp.b2, return_exact=True,
+                                 W1_scales=inp.W1_scales, W2_scales=inp.W2_scales)
+    y = run.y.double().cpu()
+    rms_col = y_ref.pow(2).mean(dim=0).sqrt()
+    err_col = (y - y_ref).abs().max(dim=0).values
+    assert bool((rms_col > 0).all())
+    worst = float((err_col / rms_col).max())
+    assert worst <= TOL_MXFP4, worst
+
+
+@pytest.mark.parametrize("x_scale", [3.0e5, 1.0e-25])
+def test_mxfp4_activation_range(x_scale):
+    # routed rows far above f16's range (|x| ~ 1e6) and far below it: the
+    # activations are quantised per 32-element block with their own E8M0
+    # scale, so any bf16 magnitude is carried (router weights scaled back so
+    # the routing is the usual one)
+    T, D, E, k, I = 300, 128, 8, 2, 128
+    base = synthetic.make_custom(T, D, E, k, I, seed=21, wfmt="mxfp4")
+    x = (base.x.float() * x_scale).to(BF16)
+    Wr = (base.Wr.float() / x_scale).to(BF16)
+    keep = ~oracle.gap_reject()(x, Wr, base.br, k)
+    x = x[keep].contiguous()
+    shape = synthetic.LayerShape("custom", x.shape[0], D, E, k, I, wfmt="mxfp4")
+    inp = dataclasses.replace(base, shape=shape, x=x, Wr=Wr).to("cuda")
+    run = _check_full(inp, TOL_MXFP4)
+    assert bool(torch.isfinite(run.y.float()).all())
 
 
 def test_empty_experts():
