@@ -85,13 +85,17 @@ typedef struct {
 } moe_dims_t;
 
 /* An expert weight tensor of logical shape (E, N, K), K the reduction dim.
- * MOE_W_BF16:  data = (E, N, K) bf16, scales = NULL.
+ * MOE_W_BF16:  data = (E, N, K) bf16, scales = NULL, prepared = NULL.
  * MOE_W_MXFP4: data = (E, N, K/2) bytes of E2M1 codes, two per byte along K
  *              with the even element in the low nibble; scales = (E, N, K/32)
- *              E8M0 bytes, value 2^(s-127), one per 32 consecutive K. */
+ *              E8M0 bytes, value 2^(s-127), one per 32 consecutive K;
+ *              prepared = NULL, or the output of moe_mxfp4_prepare() for this
+ *              weight and these dims (then the per-call preparation pass is
+ *              skipped). */
 typedef struct {
   const void* data;
   const uint8_t* scales;
+  const void* prepared;
 } moe_weight_t;
 
 /* Bytes of workspace every entry point below needs for dims d (0 if d is
@@ -196,6 +200,24 @@ MOE_API moe_status_t moe_combine(moe_dims_t d, const float* o_perm, const int32_
 MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, const uint16_t* br,
                          moe_weight_t W1, const uint16_t* b1, moe_weight_t W2, const uint16_t* b2,
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* The MXFP4 expert weights are multiplied as stored (E2M1 codes with E8M0
+ * block scales, GPT-OSS in Transformers blog, MXFP4 paragraph) on block-scaled
+ * tensor-core MMAs, which read the scales in their own layout: each MXFP4 GEMM
+ * first rewrites the scales of the experts a call routes to into that layout
+ * (and, when K is not a multiple of 128, the last 64 codes of every weight
+ * row padded to 128), into ws. The weights are static, so a caller can do it
+ * once instead: moe_mxfp4_prepare() writes the complete form for one weight
+ * (which = 1: W1 (E, 2I, D); which = 2: W2 (E, D, I)) into `out` (device
+ * memory of at least moe_mxfp4_prepared_bytes(d, which) bytes, 256-byte
+ * aligned, owned by the caller), enqueued on `stream`; pass it as that
+ * weight's moe_weight_t.prepared in every later call with the same dims
+ * (T may differ). The form depends on D, I and E only. Returns INVALID_ARG
+ * for a null pointer, a bf16 weight format or which outside {1, 2},
+ * WORKSPACE if out_bytes is too small. */
+MOE_API size_t moe_mxfp4_prepared_bytes(moe_dims_t d, int32_t which);
+MOE_API moe_status_t moe_mxfp4_prepare(moe_dims_t d, int32_t which, moe_weight_t W, void* out, size_t out_bytes,
+                               void* stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory -- e.g. code running where the memory budget is fixed up front by a

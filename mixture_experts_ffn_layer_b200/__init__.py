@@ -15,7 +15,8 @@ from ._binding import (  # noqa: F401
     MOE_W_BF16, MOE_W_MXFP4, MOE_ACT_SWIGLU, MOE_ACT_GPTOSS, EXPORTS, MoeError, Dims, dims, load, workspace_bytes,
     alloc_workspace, check_dims,
     moe_route, moe_permute, moe_gather, moe_mlp1, moe_mlp2, moe_ffn_grouped, moe_combine, moe_forward,
-    moe_read_device_status, status_str, moe_permute_noalloc, moe_selftest_wait_timeout,
+    moe_read_device_status, status_str, moe_permute_noalloc, moe_selftest_wait_timeout, mxfp4_prepared_bytes,
+    moe_mxfp4_prepare, mxfp4_prepare,
 )
 
 
@@ -39,6 +40,13 @@ class MoELayer:
         self.act, self.act_alpha, self.act_limit = act, act_alpha, act_limit
         self._ws: Optional[torch.Tensor] = None
         self._ws_T = 0
+        # MXFP4 weights: their prepare-once form (scale layout of the
+        # block-scaled MMAs), made here so that no call repeats it
+        self.W1_prepared = self.W2_prepared = None
+        if self.wfmt == MOE_W_MXFP4:
+            d1 = self.dims(1)
+            self.W1_prepared = mxfp4_prepare(d1, 1, W1, W1_scales)
+            self.W2_prepared = mxfp4_prepare(d1, 2, W2, W2_scales)
 
     def dims(self, T: int) -> Dims:
         return dims(T, self.D, self.E, self.k, self.I, self.wfmt, self.act, self.act_alpha, self.act_limit)
@@ -53,7 +61,8 @@ class MoELayer:
         T = x.shape[0]
         y = out if out is not None else torch.empty((T, self.D), dtype=torch.bfloat16, device=x.device)
         moe_forward(self.dims(T), x, self.Wr, self.br, self.W1, self.b1, self.W2, self.b2, y, self.workspace(T),
-                    W1_scales=self.W1_scales, W2_scales=self.W2_scales, stream=stream)
+                    W1_scales=self.W1_scales, W2_scales=self.W2_scales, stream=stream, W1_prepared=self.W1_prepared,
+                    W2_prepared=self.W2_prepared)
         return y
 
     __call__ = forward

@@ -24,7 +24,7 @@ STATUS = {
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_workspace_bytes", "moe_check_dims", "moe_route", "moe_permute", "moe_gather", "moe_mlp1", "moe_mlp2",
            "moe_ffn_grouped", "moe_combine", "moe_forward", "moe_read_device_status", "moe_status_str",
-           "moe_permute_noalloc", "moe_selftest_wait_timeout")
+           "moe_permute_noalloc", "moe_selftest_wait_timeout", "moe_mxfp4_prepared_bytes", "moe_mxfp4_prepare")
 
 
 class MoeError(RuntimeError):
@@ -40,7 +40,7 @@ class Dims(ctypes.Structure):
 
 
 class Weight(ctypes.Structure):
-    _fields_ = [("data", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+    _fields_ = [("data", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("prepared", ctypes.c_void_p)]
 
 
 _lib = None
@@ -74,6 +74,8 @@ def load(path: str = LIB_PATH):
         "moe_permute_noalloc": (ctypes.c_int, [Dims, VP, VP, VP, VP, VP, VP]),
         "moe_selftest_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
         "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+        "moe_mxfp4_prepared_bytes": (ctypes.c_size_t, [Dims, ctypes.c_int32]),
+        "moe_mxfp4_prepare": (ctypes.c_int, [Dims, ctypes.c_int32, Weight, VP, ctypes.c_size_t, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -97,8 +99,9 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _w(data: torch.Tensor, scales: Optional[torch.Tensor] = None) -> Weight:
-    return Weight(data.data_ptr(), None if scales is None else scales.data_ptr())
+def _w(data: torch.Tensor, scales: Optional[torch.Tensor] = None, prepared: Optional[torch.Tensor] = None) -> Weight:
+    return Weight(data.data_ptr(), None if scales is None else scales.data_ptr(),
+                  None if prepared is None else prepared.data_ptr())
 
 
 def _check(rc: int, what: str):
@@ -135,20 +138,20 @@ def moe_gather(d, x, perm, x_perm, ws, stream=None):
     _check(load().moe_gather(d, _p(x), _p(perm), _p(x_perm), _p(ws), ws.numel(), _stream(stream)), "moe_gather")
 
 
-def moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, W1_scales=None, stream=None):
-    _check(load().moe_mlp1(d, _p(x_perm), _p(offsets), _w(W1, W1_scales), _p(b1), _p(h), _p(ws), ws.numel(),
+def moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, W1_scales=None, stream=None, W1_prepared=None):
+    _check(load().moe_mlp1(d, _p(x_perm), _p(offsets), _w(W1, W1_scales, W1_prepared), _p(b1), _p(h), _p(ws), ws.numel(),
                            _stream(stream)), "moe_mlp1")
 
 
-def moe_mlp2(d, h, perm, offsets, topk_w, W2, b2, o_perm, ws, W2_scales=None, stream=None):
-    _check(load().moe_mlp2(d, _p(h), _p(perm), _p(offsets), _p(topk_w), _w(W2, W2_scales), _p(b2), _p(o_perm), _p(ws),
+def moe_mlp2(d, h, perm, offsets, topk_w, W2, b2, o_perm, ws, W2_scales=None, stream=None, W2_prepared=None):
+    _check(load().moe_mlp2(d, _p(h), _p(perm), _p(offsets), _p(topk_w), _w(W2, W2_scales, W2_prepared), _p(b2), _p(o_perm), _p(ws),
                            ws.numel(), _stream(stream)), "moe_mlp2")
 
 
 def moe_ffn_grouped(d, x, perm, offsets, topk_w, W1, b1, W2, b2, o_perm, ws, W1_scales=None, W2_scales=None,
-                    stream=None):
-    _check(load().moe_ffn_grouped(d, _p(x), _p(perm), _p(offsets), _p(topk_w), _w(W1, W1_scales), _p(b1),
-                                  _w(W2, W2_scales), _p(b2), _p(o_perm), _p(ws), ws.numel(), _stream(stream)),
+                    stream=None, W1_prepared=None, W2_prepared=None):
+    _check(load().moe_ffn_grouped(d, _p(x), _p(perm), _p(offsets), _p(topk_w), _w(W1, W1_scales, W1_prepared), _p(b1),
+                                  _w(W2, W2_scales, W2_prepared), _p(b2), _p(o_perm), _p(ws), ws.numel(), _stream(stream)),
            "moe_ffn_grouped")
 
 
@@ -156,8 +159,9 @@ def moe_combine(d, o_perm, inv, y, ws, stream=None):
     _check(load().moe_combine(d, _p(o_perm), _p(inv), _p(y), _p(ws), ws.numel(), _stream(stream)), "moe_combine")
 
 
-def moe_forward(d, x, Wr, br, W1, b1, W2, b2, y, ws, W1_scales=None, W2_scales=None, stream=None):
-    _check(load().moe_forward(d, _p(x), _p(Wr), _p(br), _w(W1, W1_scales), _p(b1), _w(W2, W2_scales), _p(b2), _p(y),
+def moe_forward(d, x, Wr, br, W1, b1, W2, b2, y, ws, W1_scales=None, W2_scales=None, stream=None, W1_prepared=None,
+                W2_prepared=None):
+    _check(load().moe_forward(d, _p(x), _p(Wr), _p(br), _w(W1, W1_scales, W1_prepared), _p(b1), _w(W2, W2_scales, W2_prepared), _p(b2), _p(y),
                               _p(ws), ws.numel(), _stream(stream)), "moe_forward")
 
 
@@ -165,6 +169,26 @@ def moe_permute_noalloc(d, topk_idx, counts, offsets, perm, inv, stream=None):
     """moe_permute without a workspace (scratch in a fixed library array)."""
     _check(load().moe_permute_noalloc(d, _p(topk_idx), _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)),
            "moe_permute_noalloc")
+
+
+def mxfp4_prepared_bytes(d, which: int) -> int:
+    return load().moe_mxfp4_prepared_bytes(d, which)
+
+
+def moe_mxfp4_prepare(d, which: int, W, W_scales, out, stream=None):
+    """The prepare-once form of an MXFP4 expert weight (which = 1: W1, 2: W2) into out."""
+    _check(load().moe_mxfp4_prepare(d, which, _w(W, W_scales), _p(out), out.numel(), _stream(stream)),
+           "moe_mxfp4_prepare")
+
+
+def mxfp4_prepare(d, which: int, W, W_scales, stream=None) -> torch.Tensor:
+    """Allocate and fill the prepare-once form of an MXFP4 expert weight."""
+    n = mxfp4_prepared_bytes(d, which)
+    if n == 0:
+        raise MoeError(2, "moe_mxfp4_prepared_bytes")
+    out = torch.empty(n, dtype=torch.uint8, device=W.device)
+    moe_mxfp4_prepare(d, which, W, W_scales, out, stream)
+    return out
 
 
 def moe_selftest_wait_timeout(ws, limit_ns: int, stream=None):

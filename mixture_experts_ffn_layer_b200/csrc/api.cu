@@ -70,8 +70,11 @@ moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes) {
 moe_status_t check_weight(const moe_dims_t& d, const moe_weight_t& w) {
   if (!w.data || !aligned32(w.data)) return MOE_ERR_INVALID_ARG;
   if (d.wfmt == MOE_W_MXFP4 && (!w.scales || !aligned32(w.scales))) return MOE_ERR_INVALID_ARG;
+  if (w.prepared && (d.wfmt != MOE_W_MXFP4 || (reinterpret_cast<uintptr_t>(w.prepared) & 255u))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+
+const uint8_t* prepared_of(const moe_weight_t& w) { return static_cast<const uint8_t*>(w.prepared); }
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -160,7 +163,7 @@ moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offse
     MOE_TRY(launch_mx_quant(d, x_perm, nullptr, d.D, offsets, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.x_sf),
                             status_word(ws), s));
     return launch_mlp1_mx(d, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.x_sf), offsets,
-                          static_cast<const uint8_t*>(W1.data), W1.scales, b1, h, nullptr, nullptr,
+                          static_cast<const uint8_t*>(W1.data), W1.scales, prepared_of(W1), b1, h, nullptr, nullptr,
                           at<uint8_t>(ws, L.mx_prep), status_word(ws), s);
   }
   const uint16_t* w1 = static_cast<const uint16_t*>(W1.data);
@@ -181,7 +184,7 @@ moe_status_t moe_mlp2(moe_dims_t d, const uint16_t* h, const int32_t* perm, cons
     MOE_TRY(launch_mx_quant(d, h, nullptr, d.I, offsets, at<uint8_t>(ws, L.hq), at<uint8_t>(ws, L.h_sf),
                             status_word(ws), s));
     return launch_mlp2_mx(d, at<uint8_t>(ws, L.hq), at<uint8_t>(ws, L.h_sf), perm, offsets, topk_w,
-                          static_cast<const uint8_t*>(W2.data), W2.scales, b2, o_perm, at<uint8_t>(ws, L.mx_prep),
+                          static_cast<const uint8_t*>(W2.data), W2.scales, prepared_of(W2), b2, o_perm, at<uint8_t>(ws, L.mx_prep),
                           status_word(ws), s);
   }
   const uint16_t* w2 = static_cast<const uint16_t*>(W2.data);
@@ -210,9 +213,9 @@ moe_status_t moe_ffn_grouped(moe_dims_t d, const uint16_t* x, const int32_t* per
     uint8_t* hq = at<uint8_t>(ws, L.hq);
     MOE_TRY(launch_mx_quant(d, x, perm, d.D, offsets, xq, at<uint8_t>(ws, L.x_sf), status_word(ws), s));
     MOE_TRY(launch_mlp1_mx(d, xq, at<uint8_t>(ws, L.x_sf), offsets, static_cast<const uint8_t*>(W1.data), W1.scales,
-                           b1, nullptr, hq, at<uint8_t>(ws, L.h_sf), at<uint8_t>(ws, L.mx_prep), status_word(ws), s));
+                           prepared_of(W1), b1, nullptr, hq, at<uint8_t>(ws, L.h_sf), at<uint8_t>(ws, L.mx_prep), status_word(ws), s));
     return launch_mlp2_mx(d, hq, at<uint8_t>(ws, L.h_sf), perm, offsets, topk_w, static_cast<const uint8_t*>(W2.data),
-                          W2.scales, b2, o_perm, at<uint8_t>(ws, L.mx_prep), status_word(ws), s);
+                          W2.scales, prepared_of(W2), b2, o_perm, at<uint8_t>(ws, L.mx_prep), status_word(ws), s);
   }
   MOE_TRY(moe_gather(d, x, perm, x_perm, ws, ws_bytes, stream));
   MOE_TRY(moe_mlp1(d, x_perm, offsets, W1, b1, h, ws, ws_bytes, stream));
@@ -247,6 +250,25 @@ moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t* Wr, co
   MOE_TRY(moe_permute(d, topk_idx, counts, offsets, perm, inv, ws, ws_bytes, stream));
   MOE_TRY(moe_ffn_grouped(d, x, perm, offsets, topk_w, W1, b1, W2, b2, o_perm, ws, ws_bytes, stream));
   return moe_combine(d, o_perm, inv, y, ws, ws_bytes, stream);
+}
+
+size_t moe_mxfp4_prepared_bytes(moe_dims_t d, int32_t which) {
+  if (moe_check_dims(d) != MOE_OK || d.wfmt != MOE_W_MXFP4 || (which != 1 && which != 2)) return 0;
+  return mx_prepared_bytes(d, which);
+}
+
+moe_status_t moe_mxfp4_prepare(moe_dims_t d, int32_t which, moe_weight_t W, void* out, size_t out_bytes,
+                               void* stream) {
+  MOE_TRY(moe_check_dims(d));
+  MOE_REQUIRE(d.wfmt == MOE_W_MXFP4 && (which == 1 || which == 2) && out);
+  MOE_REQUIRE((reinterpret_cast<uintptr_t>(out) & 255u) == 0);
+  W.prepared = nullptr;
+  MOE_TRY(check_weight(d, W));
+  const size_t need = mx_prepared_bytes(d, which);
+  if (need == 0) return MOE_ERR_UNSUPPORTED;
+  if (out_bytes < need) return MOE_ERR_WORKSPACE;
+  return mx_prepare(d, which, static_cast<const uint8_t*>(W.data), W.scales, static_cast<uint8_t*>(out),
+                    static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_read_device_status(void* ws, void* stream) {

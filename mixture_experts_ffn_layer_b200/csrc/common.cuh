@@ -107,12 +107,20 @@ size_t mx_prep_bytes(const moe_dims_t& d);
 // src rows (with perm: the gather x[perm[r] / k]) -> dst = hi (R, K) then lo (R, K), sf.
 moe_status_t launch_mx_quant(const moe_dims_t& d, const uint16_t* src, const int32_t* perm, int K,
                              const int32_t* offsets, uint8_t* dst, uint8_t* sf, int* status, cudaStream_t s);
-// mlp1 from quantised rows; h in bf16 (h non-null) or quantised for mlp2 (hq, h_sf).
+// mlp1 from quantised rows; h in bf16 (h non-null) or quantised for mlp2 (hq,
+// h_sf). prepared: the weight's prepare-once form (mx_prepare) or null, in
+// which case prep (workspace, mx_prep_bytes) receives this call's preparation.
 moe_status_t launch_mlp1_mx(const moe_dims_t& d, const uint8_t* xq, const uint8_t* x_sf, const int32_t* offsets,
-                            const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                            uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s);
+                            const uint8_t* codes, const uint8_t* scales, const uint8_t* prepared, const uint16_t* b1,
+                            uint16_t* h, uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s);
 moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_t* h_sf, const int32_t* perm,
                             const int32_t* offsets, const float* topk_w, const uint8_t* codes, const uint8_t* scales,
-                            const uint16_t* b2, float* o_perm, uint8_t* prep, int* status, cudaStream_t s);
+                            const uint8_t* prepared, const uint16_t* b2, float* o_perm, uint8_t* prep, int* status,
+                            cudaStream_t s);
+// The prepare-once form of an MXFP4 weight (which = 1: W1, 2: W2): its size
+// (0 for unsupported sizes) and the pass that writes it.
+size_t mx_prepared_bytes(const moe_dims_t& d, int which);
+moe_status_t mx_prepare(const moe_dims_t& d, int which, const uint8_t* codes, const uint8_t* scales, uint8_t* out,
+                        cudaStream_t s);
 
 }  // namespace moe

@@ -92,6 +92,7 @@ struct MxParams {
   uint8_t* hq;             // mlp1, optional: h quantised, hi (R, I) then lo (R, I) E4M3
   uint8_t* h_sf;           // and its scales, tile-blocked with h_nst stages
   int h_nst;
+  int small_max;           // experts with 1..small_max rows are left to the small-expert kernel (0: none)
 };
 
 // One stage: A hi, A lo, A scale atoms, the B operand (mma_n rows of 128
@@ -102,6 +103,25 @@ __host__ __device__ constexpr uint32_t stage_bytes(int mma_n) {
 
 __device__ __forceinline__ uint32_t sf_atom_off(int m, int kb) {
   return static_cast<uint32_t>((m & 31) * 16 + (m >> 5) * 4 + kb);
+}
+
+// Activation scales, per (m-tile g, 128-K stage q), a kSfBlock-byte block:
+//   [0, 512)     hi atom of the tile's 128 rows,
+//   [512, 1024)  lo atom,
+//   [1024, 1536) the small-expert kernel's 64-row atom of rows 0..31: line m
+//                holds row m's 4 hi scales, then its 4 lo scales (MMA rows m
+//                and 32 + m of its hi-over-lo operand).
+constexpr uint32_t kSfBlock = 2048;
+
+// Store row m's (of its 128-row tile) hi and lo scales of K block kb of a stage.
+__device__ __forceinline__ void store_act_sf(uint8_t* block, int m, int kb, uint32_t sfh, uint32_t sfl) {
+  const uint32_t o = sf_atom_off(m, kb);
+  block[o] = static_cast<uint8_t>(sfh);
+  block[512 + o] = static_cast<uint8_t>(sfl);
+  if (m < 32) {
+    block[1024 + m * 16 + kb] = static_cast<uint8_t>(sfh);
+    block[1024 + m * 16 + 4 + kb] = static_cast<uint8_t>(sfl);
+  }
 }
 
 // ---------------------------------------------------------------- E4M3 hi/lo quantisation
@@ -221,6 +241,30 @@ __device__ bool load_segments(const int32_t* offsets, int E, int64_t R, int* seg
   return !bad;
 }
 
+// Tile prefix for a kernel's schedule, by one warp: tpre[e] = sum over
+// experts e' < e of tiles(e'), with tiles(e) = per_expert(count of e).
+template <class F>
+__device__ void schedule_prefix(const int* seg, int E, int* tpre, F per_expert) {
+  const int lane = threadIdx.x & 31;
+  const int per = (E + 31) / 32;
+  const int e0 = lane * per;
+  int local = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) local += per_expert(seg[e + 1] - seg[e]);
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  int run = incl - local;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    tpre[e] = run;
+    run += per_expert(seg[e + 1] - seg[e]);
+  }
+  if (lane == 31) tpre[E] = incl;
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- quantiser kernel
 // Rows of `src` (bf16; with `perm`, row r is x[perm[r] / k], the gather of
 // the routed rows) -> hi (R, K) and lo (R, K) E4M3 at dst and dst + R*K, and
@@ -276,47 +320,87 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint16_t* __restric
     }
     const int local = static_cast<int>(r - seg[lo_e]);
     const int64_t g = mpre[lo_e] + local / BM;
-    uint8_t* atom = sf + (g * nst + b / 4) * 1024;
-    const uint32_t o = sf_atom_off(local % BM, b % 4);
-    atom[o] = static_cast<uint8_t>(sfh);
-    atom[512 + o] = static_cast<uint8_t>(sfl);
+    store_act_sf(sf + (g * nst + b / 4) * kSfBlock, local % BM, b % 4, sfh, sfl);
   }
 }
 
 // ---------------------------------------------------------------- weight preparation
-// Weight scales -> per (expert, column tile, stage) 1 KB atoms; with K % 128
-// = 64, each weight row's last 64 codes padded to a 128-element row. One
-// thread per 4 scale bytes (a row of a tile's stage) or per 16 bytes of tail.
-__global__ void __launch_bounds__(256) mx_prep_weights_kernel(const uint8_t* __restrict__ codes,
-                                                              const uint8_t* __restrict__ scales, int E, int b_rows,
-                                                              int K, int n_out, int n_tile, int mma_n, int NT,
-                                                              int nst, int swiglu, uint8_t* __restrict__ w_sf,
-                                                              uint8_t* __restrict__ tail) {
-  const int nsc = K / 32, half_k = K / 2, kfull = K / BKE * BKE;
-  const int64_t n_atoms = static_cast<int64_t>(E) * NT * nst * mma_n;
-  const int64_t n_tail = kfull < K ? static_cast<int64_t>(E) * b_rows * 4 : 0;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_atoms + n_tail;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    if (i < n_atoms) {
-      const int j = static_cast<int>(i % mma_n);
-      const int64_t tq = i / mma_n;  // (e * NT + nt) * nst + q
-      const int q = static_cast<int>(tq % nst);
-      const int64_t ent = tq / nst;
-      const int nt = static_cast<int>(ent % NT), e = static_cast<int>(ent / NT);
-      const int64_t row = static_cast<int64_t>(e) * b_rows +
-                          (swiglu ? (j < n_tile ? nt * n_tile + j : n_out + nt * n_tile + (j - n_tile))
-                                  : nt * n_tile + j);
-      const uint16_t* s2 = reinterpret_cast<const uint16_t*>(scales + row * nsc + q * 4);
-      const uint32_t lo16 = __ldg(s2);
-      const uint32_t hi16 = q * 4 + 2 < nsc ? static_cast<uint32_t>(__ldg(s2 + 1)) : 0x7f7fu;
-      *reinterpret_cast<uint32_t*>(w_sf + tq * 1024 + (j >> 7) * 512 + sf_atom_off(j & 127, 0)) = lo16 | (hi16 << 16);
-    } else {
-      const int64_t t = i - n_atoms;
-      const int64_t row = t >> 2;
-      const int piece = static_cast<int>(t & 3);
+// The weight scales in the atom layout the MMA's scale copies read, and the
+// ragged-K tail of the codes, for the experts each GEMM kernel takes:
+//  - big-tile kernel (more than small_max rows): 1 KB per (expert, column
+//    tile, stage), two atoms for the tile's mma_n weight rows;
+//  - small-expert kernel (1..small_max rows): 512 B per (expert, weight tile,
+//    stage), one atom for its 128 weight rows (mlp1: 64 gate, 64 up);
+//  - with K % 128 = 64, each weight row's last 64 codes padded with zeros to a
+//    128-element row (64 bytes), for the 4-bit TMA type.
+// With all_experts set (the prepare-once form) every expert gets both atom
+// sets and its tail rows; otherwise only what this call's routing uses.
+// One CTA per (expert, tile) or per 256 weight rows of an expert.
+struct PrepArgs {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  int E, b_rows, K, n_out, n_tile, mma_n, NT, NT2, nst, swiglu;
+  const int32_t* offsets;
+  int small_max, all_experts;
+  uint8_t* w_sf;
+  uint8_t* w_sf_small;
+  uint8_t* tail;
+};
+
+__global__ void __launch_bounds__(256) mx_prep_weights_kernel(const PrepArgs a) {
+  const int nsc = a.K / 32, half_k = a.K / 2, kfull = a.K / BKE * BKE;
+  const int64_t wrows_all = static_cast<int64_t>(a.E) * a.b_rows;
+  const int n_big = a.E * a.NT, n_small = a.small_max > 0 ? a.E * a.NT2 : 0;
+  const int rblocks = (a.b_rows + 255) / 256;
+  int blk = blockIdx.x;
+  // the 4 scale bytes of a weight row for stage q (127 = 1.0 past K or past the tensor)
+  auto sc4 = [&](int64_t row, int q) -> uint32_t {
+    if (row >= wrows_all) return 0x7f7f7f7fu;
+    const uint16_t* s2 = reinterpret_cast<const uint16_t*>(a.scales + row * nsc + q * 4);
+    const uint32_t lo16 = __ldg(s2);
+    const uint32_t hi16 = q * 4 + 2 < nsc ? static_cast<uint32_t>(__ldg(s2 + 1)) : 0x7f7fu;
+    return lo16 | (hi16 << 16);
+  };
+  auto count = [&](int e) { return a.all_experts ? -1 : __ldg(a.offsets + e + 1) - __ldg(a.offsets + e); };
+  if (blk < n_big) {
+    const int e = blk / a.NT, nt = blk - e * a.NT;
+    const int c = count(e);
+    if (!a.all_experts && c <= a.small_max) return;
+    uint8_t* out = a.w_sf + static_cast<int64_t>(blk) * a.nst * 1024;
+    for (int i = threadIdx.x; i < a.nst * a.mma_n; i += blockDim.x) {
+      const int q = i / a.mma_n, j = i - q * a.mma_n;
+      const int64_t row = static_cast<int64_t>(e) * a.b_rows +
+                          (a.swiglu ? (j < a.n_tile ? nt * a.n_tile + j : a.n_out + nt * a.n_tile + (j - a.n_tile))
+                                    : nt * a.n_tile + j);
+      *reinterpret_cast<uint32_t*>(out + q * 1024 + (j >> 7) * 512 + sf_atom_off(j & 127, 0)) = sc4(row, q);
+    }
+    return;
+  }
+  blk -= n_big;
+  if (blk < n_small) {
+    const int e = blk / a.NT2, wt = blk - e * a.NT2;
+    const int c = count(e);
+    if (!a.all_experts && (c < 1 || c > a.small_max)) return;
+    uint8_t* out = a.w_sf_small + static_cast<int64_t>(blk) * a.nst * 512;
+    for (int i = threadIdx.x; i < a.nst * 128; i += blockDim.x) {
+      const int q = i >> 7, j = i & 127;
+      const int64_t row = static_cast<int64_t>(e) * a.b_rows +
+                          (a.swiglu ? (j < 64 ? wt * 64 + j : a.n_out + wt * 64 + (j - 64)) : wt * 128 + j);
+      *reinterpret_cast<uint32_t*>(out + q * 512 + sf_atom_off(j, 0)) = sc4(row, q);
+    }
+    return;
+  }
+  blk -= n_small;
+  if (kfull < a.K) {
+    const int e = blk / rblocks, rb = blk - e * rblocks;
+    if (e >= a.E || (!a.all_experts && count(e) <= 0)) return;
+    for (int i = threadIdx.x; i < 256 * 4; i += blockDim.x) {
+      const int r = rb * 256 + (i >> 2), piece = i & 3;
+      if (r >= a.b_rows) break;
+      const int64_t row = static_cast<int64_t>(e) * a.b_rows + r;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (piece < 2) v = __ldg(reinterpret_cast<const uint4*>(codes + row * half_k + kfull / 2 + piece * 16));
-      *reinterpret_cast<uint4*>(tail + row * 64 + piece * 16) = v;
+      if (piece < 2) v = __ldg(reinterpret_cast<const uint4*>(a.codes + row * half_k + kfull / 2 + piece * 16));
+      *reinterpret_cast<uint4*>(a.tail + row * 64 + piece * 16) = v;
     }
   }
 }
@@ -337,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ctrl = ring + kStages * sst;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
   constexpr int kBars = 2 * kStages + 5;
+  static_assert(8 * kBars + 16 <= kCtrlBytes, "control block overflow");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
@@ -355,8 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- prologue: segments, tile prefixes, barriers, TMEM
   if (warp == 0) {
     const bool ok = load_segments(gp.offsets, gp.E, gp.R, seg, mpre, gp.status);
-    for (int e = lane; e <= gp.E; e += 32) tpre[e] = mpre[e] * gp.NT;
-    __syncwarp();
+    // mpre numbers the 128-row tiles of all experts (the activation scales'
+    // layout); the schedule leaves out experts the small-expert kernel takes
+    const int small_max = p.small_max, NT = gp.NT;
+    schedule_prefix(seg, gp.E, tpre, [small_max, NT](int cnt) {
+      return (cnt > small_max) ? (cnt + BM - 1) / BM * NT : 0;
+    });
     if (lane == 0) {
       *abort_flag = 0;
       *total_s = ok ? tpre[gp.E] : 0;
@@ -414,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(full_bar(s), stage_tx);
           tma_load_2d(st, &tmAhi, full_bar(s), q * BKE, row0);
           tma_load_2d(st + kAOpBytes, &tmAlo, full_bar(s), q * BKE, row0);
-          bulk_load(st + 2 * kAOpBytes, p.a_sf + (g * nst + q) * 1024, 1024, full_bar(s));
+          bulk_load(st + 2 * kAOpBytes, p.a_sf + (g * nst + q) * kSfBlock, 1024, full_bar(s));
           const CUtensorMap* tb = q < nfull ? &tmB : &tmBtail;
           const int bx = q < nfull ? q * BKE : 0;
           tma_load_2d(st + kBOff, tb, full_bar(s), bx, brow);
@@ -552,10 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int col = nt * gp.n_tile + c0;
             st_global_v8u(p.hq + row * gp.n_out + col, hi);
             st_global_v8u(p.hq + gp.R * gp.n_out + row * gp.n_out + col, lo);
-            uint8_t* atom = p.h_sf + (g * p.h_nst + col / BKE) * 1024;
-            const uint32_t o = sf_atom_off(m, (col % BKE) / 32);
-            atom[o] = static_cast<uint8_t>(sfh);
-            atom[512 + o] = static_cast<uint8_t>(sfl);
+            store_act_sf(p.h_sf + (g * p.h_nst + col / BKE) * kSfBlock, m, (col % BKE) / 32, sfh, sfl);
           }
         }
       } else {
@@ -579,15 +665,415 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- small-expert kernel
+// Experts with at most kSmallRows routed rows (decode-sized batches): the
+// weights are the MMA's M side, 128 weight rows per tile (mlp1: 64 gate rows
+// over the 64 matching up rows; mlp2: 128 output rows), and the expert's rows
+// its N side, hi rows over lo rows (N = 64), one MMA per 32-K block. Each tile
+// streams its weight rows once through a deep ring of small stages, so the
+// kernel runs at the rate HBM delivers the 4.25-bit weights.
+//   warp 0      producer, per stage: the weight codes (TMA 16U4_ALIGN16B),
+//               the expert's hi and lo rows (TMA, 32-row boxes), the weight
+//               rows' scale atom (bulk copy from the preparation pass) and the
+//               rows' 64-row scale atom (bulk copy from the activation scales);
+//   warps 1, 7  MMA: two scale copies into tensor memory and 4 block-scaled
+//               MMAs per stage; each warp takes alternate stages into its own
+//               accumulator (one warp alone issues a stage more slowly than HBM
+//               delivers it);
+//   warps 2..5  epilogue (lane = weight row): both issuers' hi + lo parts
+//               added per row in a fixed order, then SwiGLU with the up half
+//               from the other two warps via shared memory and h quantised
+//               across the warp's 32 columns, or bias * gate weight into the
+//               fp32 expert outputs.
+// Nothing here writes shared memory for the tensor core but TMA and the bulk
+// copies, so no proxy fence sits on the pipeline.
+constexpr int kSmallRows = 32;
+constexpr int kSN = 2 * kSmallRows;                  // the expert's hi rows, then its lo rows
+constexpr int kSThreads = 256;
+constexpr int kSIssuers = 2;
+constexpr int kSMma1Warp = 7;
+constexpr uint32_t kSA = 128 * 128;                  // weight operand: 128 rows x 128 B
+constexpr uint32_t kSB = kSN * 128;                  // row operand: 64 rows x 128 B
+constexpr uint32_t kSStage = kSA + kSB + 1024;       // + weight scale atom, row scale atom (512 B each)
+constexpr uint32_t kSAccStride = 64;                 // accumulator (issuer i, buffer b) at (2i + b) * 64
+constexpr uint32_t kSSfBase = 256;                   // scale regions (issuer i, r) at 256 + (2i + r) * 8
+constexpr int kSMaxStages = 8;
+constexpr int kXStride = 33;                         // floats per row of the up-half exchange buffer
+
+// Control block: 2 * stages + 9 mbarriers, then the TMEM slot, abort flag and
+// tile total (16 bytes).
+__host__ __device__ constexpr uint32_t small_ctrl_bytes(int stages) {
+  return (8u * static_cast<uint32_t>(2 * stages + 9) + 16u + 15u) / 16u * 16u;
+}
+
+struct SmallParams {
+  GemmParams g;           // E, K, n_out, b_rows, R, offsets, bias, perm, topk_w, out, status, act
+  int nst, kfull;
+  int NT2;                // weight tiles per expert
+  int stages;             // ring depth
+  const uint8_t* w_sf;    // weight scale atoms: 512 B per (expert, weight tile, stage)
+  const uint8_t* a_sf;    // activation scales, tile-blocked
+  uint8_t* hq;
+  uint8_t* h_sf;
+  int h_nst;
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// quant32's arithmetic with the 32 values spread over the warp's lanes (lane
+// i holds element i): this lane's hi and lo codes and the block's scales.
+__device__ __forceinline__ void quant32_warp(float v, uint32_t& qh, uint32_t& ql, uint32_t& sfh, uint32_t& sfl) {
+  const bool bad = __any_sync(0xffffffffu, v * 0.f != 0.f);
+  const float amax = warp_max(fabsf(v));
+  if (bad) {
+    qh = ql = 0x7fu;
+    sfh = sfl = 127;
+    return;
+  }
+  if (!(amax >= 0x1p-119f)) {
+    qh = ql = 0u;
+    sfh = sfl = 127;
+    return;
+  }
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+  const float mul = __uint_as_float(static_cast<uint32_t>(127 + 7 - e) << 23);
+  const float back = __uint_as_float(static_cast<uint32_t>(127 + e - 7) << 23);
+  sfh = static_cast<uint32_t>(e + 120);
+  qh = e4m3x2(v * mul, 0.f) & 0xffu;
+  const float r = v - e4m3x2_value(qh).x * back;
+  const float rmax = warp_max(fabsf(r));
+  if (!(rmax >= 0x1p-119f)) {
+    ql = 0u;
+    sfl = 127;
+    return;
+  }
+  const int er = static_cast<int>((__float_as_uint(rmax) >> 23) & 0xffu) - 127;
+  const float mul2 = __uint_as_float(static_cast<uint32_t>(127 + 7 - er) << 23);
+  sfl = static_cast<uint32_t>(er + 120);
+  ql = e4m3x2(r * mul2, 0.f) & 0xffu;
+}
+
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kSThreads, 1)
+    mx_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWtail,
+                    const __grid_constant__ CUtensorMap tmXhi, const __grid_constant__ CUtensorMap tmXlo,
+                    const SmallParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const GemmParams& gp = p.g;
+  const int S = p.stages;
+  uint8_t* ring = smem;
+  float* xbuf = reinterpret_cast<float*>(ring + S * kSStage);  // 64 x kXStride
+  uint8_t* ctrl = reinterpret_cast<uint8_t*>(xbuf + 64 * kXStride);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
+  const int nbars = 2 * S + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * nbars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* seg = reinterpret_cast<int*>(ctrl + small_ctrl_bytes(S));
+  int* mpre = seg + (gp.E + 1);
+  int* tpre = mpre + (gp.E + 1);
+
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (2 * S + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
+  const uint32_t xfull = bar0 + 8u * (2 * S + 5), xempty = bar0 + 8u * (2 * S + 6);  // up-half exchange
+
+  if (warp == 0) {
+    const bool ok = load_segments(gp.offsets, gp.E, gp.R, seg, mpre, gp.status);
+    const int NT2 = p.NT2;
+    schedule_prefix(seg, gp.E, tpre, [NT2](int cnt) { return (cnt >= 1 && cnt <= kSmallRows) ? NT2 : 0; });
+    if (lane == 0) {
+      *abort_flag = 0;
+      *total_s = ok ? tpre[gp.E] : 0;
+      for (int s = 0; s < S; ++s) {
+        mbar_init(full_bar(s), 1);
+        mbar_init(empty_bar(s), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(tfull(b), kSIssuers);
+        mbar_init(tempty(b), 4);
+      }
+      mbar_init(done_bar, kSIssuers);
+      mbar_init(xfull, 2);
+      mbar_init(xempty, 2);
+      fence_mbar_init();
+      if (p.kfull > 0) tma_prefetch_desc(&tmW);
+      if (p.kfull < gp.K) tma_prefetch_desc(&tmWtail);
+      tma_prefetch_desc(&tmXhi);
+      tma_prefetch_desc(&tmXlo);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_got = *tmem_slot;
+  constexpr uint32_t tmem_base = 0;
+  if (tmem_got != tmem_base && threadIdx.x == 0) record_status(gp.status, MOE_ERR_CUDA);
+  const int total = tmem_got == tmem_base ? *total_s : 0;
+  const int nst = p.nst, nfull = p.kfull / BKE;
+  // tile -> (expert, weight tile)
+  auto decode = [&](int tile, int& e, int& wt) {
+    int lo = 0, hi = gp.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tpre[mid] <= tile)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    e = lo;
+    wt = tile - tpre[e];
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      constexpr uint32_t stage_tx = 128 * (BKE / 2) + kSB + 1024;
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+        int e, wt;
+        decode(tile, e, wt);
+        const int row0 = seg[e];
+        const int64_t g = mpre[e];
+        const int64_t wr = static_cast<int64_t>(e) * gp.b_rows + (kSwiGLU ? wt * 64 : wt * 128);
+        const uint8_t* wsf = p.w_sf + (static_cast<int64_t>(e) * p.NT2 + wt) * nst * 512;
+        for (int q = 0; q < nst; ++q) {
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
+            failed = true;
+            break;
+          }
+          const uint32_t st = smem_u32(ring + s * kSStage);
+          mbar_arrive_expect_tx(full_bar(s), stage_tx);
+          const CUtensorMap* tw = q < nfull ? &tmW : &tmWtail;
+          const int wx = q < nfull ? q * BKE : 0;
+          tma_load_2d(st, tw, full_bar(s), wx, static_cast<int32_t>(wr));
+          if (kSwiGLU) tma_load_2d(st + 64 * 128, tw, full_bar(s), wx, static_cast<int32_t>(wr + gp.n_out));
+          tma_load_2d(st + kSA, &tmXhi, full_bar(s), q * BKE, row0);
+          tma_load_2d(st + kSA + kSmallRows * 128, &tmXlo, full_bar(s), q * BKE, row0);
+          bulk_load(st + kSA + kSB, wsf + q * 512, 512, full_bar(s));
+          bulk_load(st + kSA + kSB + 512, p.a_sf + (g * nst + q) * kSfBlock + 1024, 512, full_bar(s));
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (failed) {
+        record_status(gp.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        const int n = issued < S ? issued : S;  // copies still in flight
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = S - 1;
+            ph ^= 1u;
+          }
+          mbar_wait_bounded(full_bar(s), ph, nullptr, kWaitNs);
+        }
+      }
+    }
+  } else if (warp == 1 || warp == kSMma1Warp) {
+    // ------------------------------------------------------------ MMA issuers (whole warp, one lane elected)
+    // Issuer i takes the stages q = i, i + 2, ... of every tile; both track
+    // the ring position of every stage.
+    const int iss = warp == 1 ? 0 : 1;
+    const uint32_t idesc = idesc_mx(5 /* E2M1 weights */, 0 /* E4M3 rows */, kSN);
+    int s = 0, acc = 0, sfr = 0;
+    uint32_t ph = 0, pacc = 0;
+    bool failed = false;
+    for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tempty(acc), pacc ^ 1u, abort_flag, kWaitNs))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (2 * iss + acc) * kSAccStride;
+      for (int q = 0; q < nst; ++q) {
+        if ((q & 1) == iss) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs))) {
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(ring + s * kSStage);
+          const uint32_t tsf = tmem_base + kSSfBase + (2 * iss + sfr) * 8;
+          sfr ^= 1;
+          // (each copy fills 4 columns and must start on a multiple of 4)
+          tc_cp_sf_elect(tsf + 0, desc_noswizzle(st + kSA + kSB, 128));        // weight rows' scales
+          tc_cp_sf_elect(tsf + 4, desc_noswizzle(st + kSA + kSB + 512, 128));  // the 64 operand rows' scales
+          const int kleft = gp.K - q * BKE;
+          const int nkb = kleft >= BKE ? 4 : kleft / 32;
+          for (int kb = 0; kb < nkb; ++kb)
+            mma_mx_elect(d_tmem, desc_kmajor_sw128(st + kb * 32), desc_kmajor_sw128(st + kSA + kb * 32), idesc, kb,
+                         tsf + 0, tsf + 4, (q != iss || kb != 0) ? 1u : 0u);
+          tc_commit_elect(empty_bar(s));
+        }
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (failed) break;
+      tc_commit_elect(tfull(acc));  // issuer 1 with no stage (one-stage K) arrives at once
+      if (++acc == 2) {
+        acc = 0;
+        pacc ^= 1u;
+      }
+    }
+    if (failed && lane == 0) {
+      record_status(gp.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    tc_commit_elect(done_bar);
+    mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ epilogue (lane = weight row)
+    const int qd = warp & 3;  // TMEM lane quarter
+    const int m = qd * 32 + lane;
+    int acc = 0, ti = 0;
+    uint32_t pacc = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, wt;
+      decode(tile, e, wt);
+      const int row0 = seg[e], cnt = seg[e + 1] - seg[e];
+      const bool ok = mbar_wait_bounded(tfull(acc), pacc, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          record_status(gp.status, MOE_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kSAccStride;
+      // row t's value: issuer 0's (hi + lo) part, plus issuer 1's when the
+      // tile had a second stage, added in that order
+      float v[kSmallRows];
+      {
+        uint32_t hv[32], lv[32];
+        tmem_ld_x32(tb, hv);
+        tmem_ld_x32(tb + kSmallRows, lv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < kSmallRows; ++t) v[t] = __uint_as_float(hv[t]) + __uint_as_float(lv[t]);
+        if (nst > 1) {
+          tmem_ld_x32(tb + 2 * kSAccStride, hv);
+          tmem_ld_x32(tb + 2 * kSAccStride + kSmallRows, lv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < kSmallRows; ++t) v[t] += __uint_as_float(hv[t]) + __uint_as_float(lv[t]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(acc));  // the accumulator is in registers now
+      if (++acc == 2) {
+        acc = 0;
+        pacc ^= 1u;
+      }
+      if (kSwiGLU) {
+        // lanes 64..127 hold the up half: hand it to the gate warps through
+        // shared memory (bounded waits on two mbarriers, one phase per tile)
+        bool xok = true;
+        if (qd >= 2) {
+          xok = __all_sync(0xffffffffu, mbar_wait_bounded(xempty, (ti & 1) ^ 1u, abort_flag, kWaitNs));
+          if (xok) {
+#pragma unroll
+            for (int t = 0; t < kSmallRows; ++t) xbuf[(m - 64) * kXStride + t] = v[t];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xfull);
+          }
+        } else {
+          xok = __all_sync(0xffffffffu, mbar_wait_bounded(xfull, ti & 1, abort_flag, kWaitNs));
+          if (xok) {
+            const int col = wt * 64 + m;  // h column
+            const float bg = bf16_bits_to_float(gp.bias[static_cast<int64_t>(e) * gp.b_rows + col]);
+            const float bu = bf16_bits_to_float(gp.bias[static_cast<int64_t>(e) * gp.b_rows + gp.n_out + col]);
+            const int64_t g = mpre[e];
+            const int col0 = wt * 64 + qd * 32;  // the warp's 32-column scale block
+            float u[kSmallRows];
+#pragma unroll
+            for (int t = 0; t < kSmallRows; ++t) u[t] = xbuf[m * kXStride + t];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xempty);
+#pragma unroll
+            for (int t = 0; t < kSmallRows; ++t) {
+              if (t >= cnt) break;  // warp-uniform
+              const float hb = bf16_bits_to_float(float_to_bf16_bits(glu_act(v[t] + bg, u[t] + bu, gp.act)));
+              const int64_t r = row0 + t;
+              if (p.hq != nullptr) {
+                uint32_t qh, ql, sfh, sfl;
+                quant32_warp(hb, qh, ql, sfh, sfl);
+                p.hq[r * gp.n_out + col] = static_cast<uint8_t>(qh);
+                p.hq[gp.R * gp.n_out + r * gp.n_out + col] = static_cast<uint8_t>(ql);
+                if (lane == 0)
+                  store_act_sf(p.h_sf + (g * p.h_nst + col0 / BKE) * kSfBlock, t, (col0 % BKE) / 32, sfh, sfl);
+              } else {
+                static_cast<uint16_t*>(gp.out)[r * gp.n_out + col] = float_to_bf16_bits(hb);
+              }
+            }
+          }
+        }
+        if (!xok) {
+          if (lane == 0) {
+            record_status(gp.status, MOE_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        ++ti;
+      } else {
+        const int col = wt * 128 + m;  // output column
+        if (col < gp.n_out) {
+          const float bb = bf16_bits_to_float(gp.bias[static_cast<int64_t>(e) * gp.b_rows + col]);
+#pragma unroll
+          for (int t = 0; t < kSmallRows; ++t) {
+            if (t >= cnt) break;
+            const int64_t r = row0 + t;
+            const int32_t a = gp.perm[r];
+            float wgt = 0.f;
+            if (a >= 0 && a < gp.R)
+              wgt = gp.topk_w[a];
+            else
+              record_status(gp.status, MOE_ERR_DEVICE_BOUNDS);
+            static_cast<float*>(gp.out)[r * gp.n_out + col] = wgt * (v[t] + bb);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_got, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
-// (rows, inner) bytes, loaded as 128 x 128-byte boxes with the 128-byte
+// (rows, inner) bytes, loaded as 128-byte x box_rows boxes with the 128-byte
 // swizzle (the K-major E4M3 operand layout).
-bool make_tmap_e4m3(CUtensorMap* map, const uint8_t* base, uint64_t inner, uint64_t rows) {
+bool make_tmap_e4m3(CUtensorMap* map, const uint8_t* base, uint64_t inner, uint64_t rows, uint32_t box_rows = BM) {
   auto fn = tma_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), static_cast<cuuint32_t>(BM)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -629,32 +1115,121 @@ int pick_tile(int n, int max_tile, int step) {
 int mlp1_ntile(const moe_dims_t& d) { return pick_tile(d.I, kMaxN / 2 / 32 * 32, 32); }
 int mlp2_ntile(const moe_dims_t& d) { return pick_tile(d.D, kMaxN, 16); }
 
-size_t w_sf_bytes(int E, int NT, int K) { return static_cast<size_t>(E) * NT * ((K + BKE - 1) / BKE) * 1024; }
-size_t w_tail_bytes(int E, int b_rows, int K) { return K % BKE ? static_cast<size_t>(E) * b_rows * 64 : 0; }
+
+size_t small_smem_bytes(int stages, int E) {
+  return 1024 + static_cast<size_t>(stages) * kSStage + 64 * kXStride * sizeof(float) + small_ctrl_bytes(stages) +
+         3 * static_cast<size_t>(E + 1) * sizeof(int);
+}
+
+// The preparation region of one GEMM: big-tile atoms, small-tile atoms, tail rows.
+struct PrepLayout {
+  size_t big, small, tail, total;
+};
+PrepLayout prep_layout(int E, int b_rows, int K, int NT, int NT2) {
+  PrepLayout L{};
+  const int nst = (K + BKE - 1) / BKE;
+  L.big = 0;
+  L.small = align_up(static_cast<size_t>(E) * NT * nst * 1024, 256);
+  L.tail = L.small + align_up(static_cast<size_t>(E) * NT2 * nst * 512, 256);
+  L.total = L.tail + (K % BKE ? align_up(static_cast<size_t>(E) * b_rows * 64, 256) : 0);
+  return L;
+}
+
+// One grouped GEMM with MXFP4 weights: the preparation pass, then the
+// small-expert kernel (experts with 1..kSmallRows rows) and the big-tile
+// kernel (the others), each skipping the other's experts.
+// The small-expert kernel's geometry for a GEMM: weight tiles per expert,
+// ring depth, and whether it runs at all (else every expert takes big tiles).
+struct SmallGeom {
+  int NT2, stages;
+  bool ok;
+};
+template <bool kSwiGLU>
+SmallGeom small_geom(const GemmParams& g) {
+  SmallGeom sg{};
+  sg.NT2 = kSwiGLU ? g.n_out / 64 : (g.n_out + 127) / 128;
+  sg.stages = kSMaxStages;
+  while (sg.stages >= 3 && small_smem_bytes(sg.stages, g.E) > 227 * 1024) --sg.stages;
+  sg.ok = sg.stages >= 3 && (!kSwiGLU || g.n_out % 64 == 0);
+  return sg;
+}
+
+// The preparation pass into `out` for the given routing (offsets) or, with
+// all_experts, for every expert (the prepare-once form).
+template <bool kSwiGLU>
+moe_status_t run_prep(const MxParams& p, const uint8_t* codes, const uint8_t* scales, uint8_t* out, bool all_experts,
+                      cudaStream_t s) {
+  const GemmParams& g = p.g;
+  const SmallGeom sg = small_geom<kSwiGLU>(g);
+  const PrepLayout L = prep_layout(g.E, g.b_rows, g.K, g.NT, sg.NT2);
+  PrepArgs pa{codes, scales, g.E, g.b_rows, g.K, g.n_out, g.n_tile, g.mma_n, g.NT, sg.NT2, p.nst, kSwiGLU ? 1 : 0,
+              g.offsets, sg.ok ? kSmallRows : 0, all_experts ? 1 : 0, out + L.big, out + L.small, out + L.tail};
+  const int blocks = g.E * g.NT + (sg.ok ? g.E * sg.NT2 : 0) + (g.K % BKE ? g.E * ((g.b_rows + 255) / 256) : 0);
+  mx_prep_weights_kernel<<<blocks, 256, 0, s>>>(pa);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 template <bool kSwiGLU>
+size_t prep_bytes(const MxParams& p) {
+  return prep_layout(p.g.E, p.g.b_rows, p.g.K, p.g.NT, small_geom<kSwiGLU>(p.g).NT2).total;
+}
+
+// prep: the preparation region, written here per call (only what this call's
+// routing uses) unless `prepared` says it already holds the prepare-once form.
+template <bool kSwiGLU>
 moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8_t* scales, uint8_t* prep,
-                            MxParams p, cudaStream_t s) {
+                            bool prepared, MxParams p, cudaStream_t s) {
   const GemmParams& g = p.g;
-  // weight scales into per-stage atoms (and the ragged-K tail rows) in prep
-  uint8_t* w_sf = prep;
-  uint8_t* tail = prep + align_up(w_sf_bytes(g.E, g.NT, g.K), 256);
-  {
-    const int64_t n = static_cast<int64_t>(g.E) * g.NT * p.nst * g.mma_n +
-                      (g.K % BKE ? static_cast<int64_t>(g.E) * g.b_rows * 4 : 0);
-    const int64_t blocks = (n + 255) / 256;
-    const int grid = static_cast<int>(blocks < 8 * num_sms() ? blocks : 8 * num_sms());
-    mx_prep_weights_kernel<<<grid, 256, 0, s>>>(codes, scales, g.E, g.b_rows, g.K, g.n_out, g.n_tile, g.mma_n, g.NT,
-                                                p.nst, kSwiGLU ? 1 : 0, w_sf, tail);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  p.kfull = g.K / BKE * BKE;
+  const SmallGeom sg = small_geom<kSwiGLU>(g);
+  SmallParams sp{};
+  sp.g = g;
+  sp.nst = p.nst;
+  sp.kfull = p.kfull;
+  sp.NT2 = sg.NT2;
+  sp.stages = sg.stages;
+  const bool small_ok = sg.ok;
+  p.small_max = small_ok ? kSmallRows : 0;
+  const PrepLayout L = prep_layout(g.E, g.b_rows, g.K, g.NT, sp.NT2);
+  uint8_t* w_sf = prep + L.big;
+  uint8_t* w_sf_small = prep + L.small;
+  uint8_t* tail = prep + L.tail;
+  if (!prepared) {
+    const moe_status_t st = run_prep<kSwiGLU>(p, codes, scales, prep, false, s);
+    if (st != MOE_OK) return st;
   }
   p.w_sf = w_sf;
-  p.kfull = g.K / BKE * BKE;
+  sp.w_sf = w_sf_small;
+  sp.a_sf = p.a_sf;
+  sp.hq = p.hq;
+  sp.h_sf = p.h_sf;
+  sp.h_nst = p.h_nst;
+  const uint64_t wrows = static_cast<uint64_t>(g.E) * g.b_rows;
+  const uint8_t* alo = aq + g.R * g.K;
+
+  if (small_ok) {
+    CUtensorMap tw, twt, txh, txl;
+    memset(&tw, 0, sizeof(tw));
+    memset(&twt, 0, sizeof(twt));
+    const uint32_t wbox = kSwiGLU ? 64 : 128;
+    if (p.kfull > 0 && !make_tmap_e2m1(&tw, codes, p.kfull, g.K / 2, wrows, wbox)) return MOE_ERR_CUDA;
+    if (p.kfull < g.K && !make_tmap_e2m1(&twt, tail, BKE, 64, wrows, wbox)) return MOE_ERR_CUDA;
+    if (!make_tmap_e4m3(&txh, aq, g.K, g.R, kSmallRows) || !make_tmap_e4m3(&txl, alo, g.K, g.R, kSmallRows))
+      return MOE_ERR_CUDA;
+    const size_t smem = small_smem_bytes(sp.stages, g.E);
+    if (cudaFuncSetAttribute(mx_small_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int64_t max_tiles = static_cast<int64_t>(g.E) * sp.NT2;
+    const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
+    mx_small_kernel<kSwiGLU><<<grid, kSThreads, smem, s>>>(tw, twt, txh, txl, sp);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
   CUtensorMap thi, tlo, tb, tt;
   memset(&tb, 0, sizeof(tb));
   memset(&tt, 0, sizeof(tt));
-  if (!make_tmap_e4m3(&thi, aq, g.K, g.R) || !make_tmap_e4m3(&tlo, aq + g.R * g.K, g.K, g.R)) return MOE_ERR_CUDA;
-  const uint64_t wrows = static_cast<uint64_t>(g.E) * g.b_rows;
+  if (!make_tmap_e4m3(&thi, aq, g.K, g.R) || !make_tmap_e4m3(&tlo, alo, g.K, g.R)) return MOE_ERR_CUDA;
   const uint32_t box_rows = static_cast<uint32_t>(kSwiGLU ? g.n_tile : g.mma_n);
   if (p.kfull > 0 && !make_tmap_e2m1(&tb, codes, p.kfull, g.K / 2, wrows, box_rows)) return MOE_ERR_CUDA;
   if (p.kfull < g.K && !make_tmap_e2m1(&tt, tail, BKE, 64, wrows, box_rows)) return MOE_ERR_CUDA;
@@ -673,14 +1248,12 @@ moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8
 
 size_t mx_sf_bytes(const moe_dims_t& d, int K) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
-  return static_cast<size_t>((R + BM - 1) / BM + d.E) * ((K + BKE - 1) / BKE) * 1024;
+  return static_cast<size_t>((R + BM - 1) / BM + d.E) * ((K + BKE - 1) / BKE) * kSfBlock;
 }
 
 size_t mx_prep_bytes(const moe_dims_t& d) {
-  const int n1 = mlp1_ntile(d), n2 = mlp2_ntile(d);
-  if (n1 == 0 || n2 == 0) return 0;
-  const size_t p1 = align_up(w_sf_bytes(d.E, d.I / n1, d.D), 256) + w_tail_bytes(d.E, 2 * d.I, d.D);
-  const size_t p2 = align_up(w_sf_bytes(d.E, d.D / n2, d.I), 256) + w_tail_bytes(d.E, d.D, d.I);
+  const size_t p1 = mx_prepared_bytes(d, 1), p2 = mx_prepared_bytes(d, 2);
+  if (p1 == 0 || p2 == 0) return 0;
   return align_up(p1 > p2 ? p1 : p2, 256);
 }
 
@@ -694,58 +1267,87 @@ moe_status_t launch_mx_quant(const moe_dims_t& d, const uint16_t* src, const int
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status_t launch_mlp1_mx(const moe_dims_t& d, const uint8_t* xq, const uint8_t* x_sf, const int32_t* offsets,
-                            const uint8_t* codes, const uint8_t* scales, const uint16_t* b1, uint16_t* h,
-                            uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s) {
-  const int nh = mlp1_ntile(d);
-  if (nh == 0) return MOE_ERR_UNSUPPORTED;
+MxParams mlp1_params(const moe_dims_t& d) {
   MxParams p{};
   GemmParams& g = p.g;
   g.E = d.E;
   g.K = d.D;
   g.n_out = d.I;
-  g.n_tile = nh;
-  g.mma_n = 2 * nh;
-  g.NT = d.I / nh;
+  g.n_tile = mlp1_ntile(d);
+  g.mma_n = 2 * g.n_tile;
+  g.NT = g.n_tile ? d.I / g.n_tile : 0;
   g.b_rows = 2 * d.I;
   g.R = static_cast<int64_t>(d.T) * d.k;
-  g.offsets = offsets;
-  g.bias = b1;
   g.act = act_of(d);
-  g.out = h;
-  g.status = status;
   p.nst = (d.D + BKE - 1) / BKE;
-  p.a_sf = x_sf;
-  p.hq = hq;
-  p.h_sf = h_sf;
   p.h_nst = (d.I + BKE - 1) / BKE;
-  return launch_mx_gemm<true>(xq, codes, scales, prep, p, s);
+  return p;
 }
 
-moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_t* h_sf, const int32_t* perm,
-                            const int32_t* offsets, const float* topk_w, const uint8_t* codes, const uint8_t* scales,
-                            const uint16_t* b2, float* o_perm, uint8_t* prep, int* status, cudaStream_t s) {
-  const int nt = mlp2_ntile(d);
-  if (nt == 0) return MOE_ERR_UNSUPPORTED;
+MxParams mlp2_params(const moe_dims_t& d) {
   MxParams p{};
   GemmParams& g = p.g;
   g.E = d.E;
   g.K = d.I;
   g.n_out = d.D;
-  g.n_tile = nt;
-  g.mma_n = nt;
-  g.NT = d.D / nt;
+  g.n_tile = mlp2_ntile(d);
+  g.mma_n = g.n_tile;
+  g.NT = g.n_tile ? d.D / g.n_tile : 0;
   g.b_rows = d.D;
   g.R = static_cast<int64_t>(d.T) * d.k;
-  g.offsets = offsets;
-  g.bias = b2;
-  g.perm = perm;
-  g.topk_w = topk_w;
-  g.out = o_perm;
-  g.status = status;
   p.nst = (d.I + BKE - 1) / BKE;
+  return p;
+}
+
+moe_status_t launch_mlp1_mx(const moe_dims_t& d, const uint8_t* xq, const uint8_t* x_sf, const int32_t* offsets,
+                            const uint8_t* codes, const uint8_t* scales, const uint8_t* prepared, const uint16_t* b1,
+                            uint16_t* h, uint8_t* hq, uint8_t* h_sf, uint8_t* prep, int* status, cudaStream_t s) {
+  MxParams p = mlp1_params(d);
+  if (p.g.n_tile == 0) return MOE_ERR_UNSUPPORTED;
+  p.g.offsets = offsets;
+  p.g.bias = b1;
+  p.g.out = h;
+  p.g.status = status;
+  p.a_sf = x_sf;
+  p.hq = hq;
+  p.h_sf = h_sf;
+  return launch_mx_gemm<true>(xq, codes, scales, prepared ? const_cast<uint8_t*>(prepared) : prep, prepared != nullptr,
+                              p, s);
+}
+
+moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_t* h_sf, const int32_t* perm,
+                            const int32_t* offsets, const float* topk_w, const uint8_t* codes, const uint8_t* scales,
+                            const uint8_t* prepared, const uint16_t* b2, float* o_perm, uint8_t* prep, int* status,
+                            cudaStream_t s) {
+  MxParams p = mlp2_params(d);
+  if (p.g.n_tile == 0) return MOE_ERR_UNSUPPORTED;
+  p.g.offsets = offsets;
+  p.g.bias = b2;
+  p.g.perm = perm;
+  p.g.topk_w = topk_w;
+  p.g.out = o_perm;
+  p.g.status = status;
   p.a_sf = h_sf;
-  return launch_mx_gemm<false>(hq, codes, scales, prep, p, s);
+  return launch_mx_gemm<false>(hq, codes, scales, prepared ? const_cast<uint8_t*>(prepared) : prep, prepared != nullptr,
+                               p, s);
+}
+
+size_t mx_prepared_bytes(const moe_dims_t& d, int which) {
+  if (which == 1) {
+    const MxParams p = mlp1_params(d);
+    return p.g.n_tile ? prep_bytes<true>(p) : 0;
+  }
+  if (which == 2) {
+    const MxParams p = mlp2_params(d);
+    return p.g.n_tile ? prep_bytes<false>(p) : 0;
+  }
+  return 0;
+}
+
+moe_status_t mx_prepare(const moe_dims_t& d, int which, const uint8_t* codes, const uint8_t* scales, uint8_t* out,
+                        cudaStream_t s) {
+  if (which == 1) return run_prep<true>(mlp1_params(d), codes, scales, out, true, s);
+  return run_prep<false>(mlp2_params(d), codes, scales, out, true, s);
 }
 
 }  // namespace moe

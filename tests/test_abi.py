@@ -64,12 +64,14 @@ def test_workspace_bytes_cover_the_decode_paths():
     assert base + splits * T * E * 4 <= n <= base + splits * T * E * 4 + 1024 * 1024
     nq = moe.workspace_bytes(moe.dims(T, D, E, k, I, wfmt=moe.MOE_W_MXFP4))
     mtiles = -(-R // 128) + E
-    sf = mtiles * -(-D // 128) * 1024 + mtiles * -(-I // 128) * 1024
-    # the weights' scales as per-stage atoms (E x 30 column tiles x 23 stages
-    # x 1 KB for mlp1) and the padded last 64 codes of every mlp1 weight row
-    prep = E * (I // 96) * -(-D // 128) * 1024 + E * 2 * I * 64
+    sf = mtiles * -(-D // 128) * 2048 + mtiles * -(-I // 128) * 2048  # 2 KB of scales per (128-row tile, 128-K stage)
+    # the weights' scales in the MMA's atom layout for both kernels (mlp1: E x
+    # 30 column tiles x 23 stages x 1 KB, E x 45 weight tiles x 23 stages x
+    # 512 B) and the padded last 64 codes of every mlp1 weight row
+    nst = -(-D // 128)
+    prep = E * (I // 96) * nst * 1024 + E * (I // 64) * nst * 512 + E * 2 * I * 64
     assert R * (D + I) * 2 + sf + prep <= nq - n <= R * (D + I) * 2 + sf + prep + 8192
-    assert nq - n < 64 * 1024 * 1024  # no expanded weights (1.59 GB at this shape)
+    assert nq - n < 128 * 1024 * 1024  # no expanded weights (1.59 GB at this shape)
 
 
 def test_workspace_bytes_covers_intermediates():
@@ -80,7 +82,7 @@ def test_workspace_bytes_covers_intermediates():
     assert need <= n <= need + 4 * 1024 * 1024
     dq = moe.dims(8192, 2880, 32, 4, 2880, wfmt=moe.MOE_W_MXFP4)
     extra = moe.workspace_bytes(dq) - n
-    assert R * 2880 * 4 <= extra <= R * 2880 * 4 + 64 * 1024 * 1024  # hi/lo operands + scales, no weight copies
+    assert R * 2880 * 4 <= extra <= R * 2880 * 4 + 128 * 1024 * 1024  # hi/lo operands + scales, no weight copies
     with pytest.raises(moe.MoeError):
         moe.workspace_bytes(moe.dims(8, 64, 4, 5, 64))
 
@@ -163,3 +165,32 @@ def test_noalloc_permute_size_limit_boundary():
     # invalid dims are refused by the dims check first
     assert lib.moe_permute_noalloc(moe.dims(8, 64, 4, 5, 64), *[vp(ar.base)] * 5, None) == 1
     assert lib.moe_permute_noalloc(moe.dims(8, 64, 4, 2, 64), None, *[vp(ar.base)] * 4, None) == 1
+
+
+def test_mxfp4_prepare_arguments():
+    # the prepare-once form of an MXFP4 weight: sizes for each weight, and
+    # synchronous refusals (bf16 weights, an unknown weight, a null pointer,
+    # a short buffer, a prepared form on a bf16 call)
+    lib = moe.load()
+    dq = moe.dims(64, 2880, 32, 4, 2880, wfmt=moe.MOE_W_MXFP4)
+    n1, n2 = moe.mxfp4_prepared_bytes(dq, 1), moe.mxfp4_prepared_bytes(dq, 2)
+    nst = -(-2880 // 128)
+    assert n1 >= 32 * 30 * nst * 1024 + 32 * 45 * nst * 512 + 32 * 5760 * 64
+    assert n2 >= 32 * 12 * nst * 1024 + 32 * 23 * nst * 512 + 32 * 2880 * 64
+    assert moe.mxfp4_prepared_bytes(moe.dims(64, 2880, 32, 4, 2880), 1) == 0  # bf16 weights
+    assert moe.mxfp4_prepared_bytes(dq, 3) == 0
+    ar = _Arena(96 << 20)
+    vp = ctypes.c_void_p
+    w = _binding.Weight(ar.take(), ar.take(), None)
+    out = vp(ar.take(n1))
+    assert lib.moe_mxfp4_prepare(moe.dims(64, 2880, 32, 4, 2880), 1, w, out, n1, None) == 1
+    assert lib.moe_mxfp4_prepare(dq, 3, w, out, n1, None) == 1
+    assert lib.moe_mxfp4_prepare(dq, 1, w, None, n1, None) == 1
+    assert lib.moe_mxfp4_prepare(dq, 1, w, vp(ar.take() + 32), n1, None) == 1  # not 256-byte aligned
+    assert lib.moe_mxfp4_prepare(dq, 1, _binding.Weight(ar.take(), None, None), out, n1, None) == 1  # no scales
+    assert lib.moe_mxfp4_prepare(dq, 1, w, out, n1 - 1, None) == 3
+    d = moe.dims(64, 64, 4, 2, 64)
+    ws_n = moe.workspace_bytes(d)
+    ws = vp(ar.take(ws_n))
+    wp = _binding.Weight(ar.take(), None, ar.take())  # prepared form on bf16 weights
+    assert lib.moe_mlp1(d, vp(ar.take()), vp(ar.take()), wp, vp(ar.take()), vp(ar.take()), ws, ws_n, None) == 1

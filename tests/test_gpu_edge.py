@@ -10,7 +10,7 @@ import torch
 import mixture_experts_ffn_layer_b200 as moe
 import oracle
 import synthetic
-from helpers import TOL_BF16, TOL_MXFP4, assert_close_rms, run_forward, run_stages
+from helpers import TOL_BF16, TOL_MXFP4, assert_close_rms, dims_of, run_forward, run_stages
 
 pytestmark = pytest.mark.gpu
 
@@ -109,6 +109,41 @@ def test_forward_mxfp4_matches_stages(T, D, E, k, I):
     y2 = run_forward(inp)
     assert torch.equal(y1.view(torch.int16), run.y.view(torch.int16))
     assert torch.equal(y2.view(torch.int16), y1.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,D,E,k,I", [
+    (64, 2880, 32, 4, 2880),  # decode-sized: the small-expert kernel
+    (600, 128, 4, 2, 192),    # several 128-row tiles per expert: the big-tile kernel
+    (300, 192, 16, 2, 320),   # both kernels in one call (hot and cold experts), ragged K
+])
+def test_mxfp4_prepared_weights_match_per_call(T, D, E, k, I):
+    # weights prepared once (moe_mxfp4_prepare) give bitwise the result of the
+    # per-call preparation, through the staged and the one-call entry points
+    inp = synthetic.make_custom(T, D, E, k, I, seed=T + 5 * E, device="cuda", wfmt="mxfp4", reject=oracle.gap_reject())
+    if T == 300:
+        br = torch.zeros(E)
+        br[2] = 3.0
+        inp.br = br.to(BF16).to("cuda")
+    run = run_stages(inp)
+    assert run.status == 0
+    d = dims_of(inp)
+    p1 = moe.mxfp4_prepare(d, 1, inp.W1, inp.W1_scales)
+    p2 = moe.mxfp4_prepare(d, 2, inp.W2, inp.W2_scales)
+    s = inp.shape
+    ws = moe.alloc_workspace(d)
+    h = torch.empty((s.T * s.k, s.I), dtype=BF16, device="cuda")
+    o = torch.empty((s.T * s.k, s.D), dtype=torch.float32, device="cuda")
+    moe.moe_mlp1(d, run.x_perm, run.offsets, inp.W1, inp.b1, h, ws, W1_scales=inp.W1_scales, W1_prepared=p1)
+    moe.moe_mlp2(d, h, run.perm, run.offsets, run.topk_w, inp.W2, inp.b2, o, ws, W2_scales=inp.W2_scales,
+                 W2_prepared=p2)
+    assert moe.moe_read_device_status(ws) == 0
+    assert torch.equal(h.view(torch.int16), run.h.view(torch.int16))
+    assert torch.equal(o, run.o_perm)
+    y = torch.empty((s.T, s.D), dtype=BF16, device="cuda")
+    moe.moe_forward(d, inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws, W1_scales=inp.W1_scales,
+                    W2_scales=inp.W2_scales, W1_prepared=p1, W2_prepared=p2)
+    assert moe.moe_read_device_status(ws) == 0
+    assert torch.equal(y.view(torch.int16), run.y.view(torch.int16))
 
 
 @pytest.mark.parametrize("T", [40, 700])
