@@ -90,8 +90,9 @@ typedef struct {
  *              with the even element in the low nibble; scales = (E, N, K/32)
  *              E8M0 bytes, value 2^(s-127), one per 32 consecutive K;
  *              prepared = NULL, or the output of moe_mxfp4_prepare() for this
- *              weight and these dims (then the per-call preparation pass is
- *              skipped). */
+ *              weight and these dims: the GEMMs then read only the prepared
+ *              copy (no per-call preparation pass), and data and scales may
+ *              be NULL. */
 typedef struct {
   const void* data;
   const uint8_t* scales;
@@ -207,7 +208,13 @@ MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t
  * first rewrites the scales of the experts a call routes to into that layout
  * (and, when K is not a multiple of 128, the last 64 codes of every weight
  * row padded to 128), into ws. The weights are static, so a caller can do it
- * once instead: moe_mxfp4_prepare() writes the complete form for one weight
+ * once instead, which also stores the codes K-block-major -- for each block
+ * of 128 K, every row's 64 code bytes side by side, the ragged last block
+ * padded with zeros -- so the GEMMs read them as contiguous runs rather than
+ * as 64-byte pieces of rows K/2 bytes apart (about twice the delivered HBM
+ * bandwidth on decode-sized batches). The form takes about the size of the
+ * codes plus 1.5x the scales; once it exists, the original data and scales
+ * are not read again. moe_mxfp4_prepare() writes the complete form for one weight
  * (which = 1: W1 (E, 2I, D); which = 2: W2 (E, D, I)) into `out` (device
  * memory of at least moe_mxfp4_prepared_bytes(d, which) bytes, 256-byte
  * aligned, owned by the caller), enqueued on `stream`; pass it as that

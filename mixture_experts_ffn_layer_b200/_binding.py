@@ -99,8 +99,10 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _w(data: torch.Tensor, scales: Optional[torch.Tensor] = None, prepared: Optional[torch.Tensor] = None) -> Weight:
-    return Weight(data.data_ptr(), None if scales is None else scales.data_ptr(),
+def _w(data: Optional[torch.Tensor], scales: Optional[torch.Tensor] = None,
+       prepared: Optional[torch.Tensor] = None) -> Weight:
+    # (data and scales may be None next to an MXFP4 prepared form)
+    return Weight(None if data is None else data.data_ptr(), None if scales is None else scales.data_ptr(),
                   None if prepared is None else prepared.data_ptr())
 
 

@@ -68,9 +68,15 @@ moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes) {
 }
 
 moe_status_t check_weight(const moe_dims_t& d, const moe_weight_t& w) {
+  if (w.prepared) {
+    // the prepare-once form holds everything the MXFP4 GEMMs read: data and
+    // scales may be null
+    if (d.wfmt != MOE_W_MXFP4 || (reinterpret_cast<uintptr_t>(w.prepared) & 255u)) return MOE_ERR_INVALID_ARG;
+    if ((w.data && !aligned32(w.data)) || (w.scales && !aligned32(w.scales))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+  }
   if (!w.data || !aligned32(w.data)) return MOE_ERR_INVALID_ARG;
   if (d.wfmt == MOE_W_MXFP4 && (!w.scales || !aligned32(w.scales))) return MOE_ERR_INVALID_ARG;
-  if (w.prepared && (d.wfmt != MOE_W_MXFP4 || (reinterpret_cast<uintptr_t>(w.prepared) & 255u))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 

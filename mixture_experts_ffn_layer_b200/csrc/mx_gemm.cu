@@ -22,12 +22,13 @@
 // One persistent, warp-specialised kernel for mlp1 (+bias, SwiGLU) and mlp2
 // (+bias, gate weight); tiles are (expert, column tile, 128-row tile) over
 // the device-side expert offsets, as in the bf16 grouped GEMM:
-//   warp 0      producer, per 128-K stage: the tile's 128 activation rows as
-//               hi and lo E4M3 boxes (TMA, 128-byte swizzle) and their 1 KB of
-//               scale factors (bulk copy); the weight rows' E2M1 codes (TMA
-//               with the 16U4_ALIGN16B type, which unpacks every 8 bytes of
-//               codes into the 16-byte slot the MMA's E2M1 operand layout
-//               wants) and their 1 KB of scale factors (bulk copy);
+//   warp 0      activation-side producer, per 128-K stage: the tile's 128
+//               rows, hi and lo E4M3 planes in one 3-D TMA box (128-byte
+//               swizzle), and their 1 KB of scale factors (TMA);
+//   warp 6      weight-side producer: the weight rows' E2M1 codes, gate and
+//               up halves in one TMA box of the 16U4_ALIGN16B type (which
+//               unpacks every 8 bytes of codes into the 16-byte slot the MMA's
+//               E2M1 operand layout wants), and their 1 KB of scale factors;
 //   warp 1      MMA: tcgen05.cp of the stage's scale factors into tensor
 //               memory, then per 32-K block two block-scaled MMAs (hi, lo),
 //               M = 128 rows, N = the tile's weight rows; whole warp, one
@@ -35,21 +36,31 @@
 //   warps 2..5  epilogue: bias + SwiGLU into h (bf16, or straight into the
 //               quantised hi/lo form mlp2 reads), or bias * gate weight into
 //               the fp32 expert outputs.
+// A thread that issues a TMA copy cannot issue the next for ~60 ns whatever
+// its size, so each operand of a stage is one copy and two threads share the
+// copies; each completes its own full barrier, and the MMA warp waits on both.
 //
 // Scale factors reach tensor memory through tcgen05.cp, which reads 128 rows'
 // scales of 4 K blocks as a 32 x 16-byte shared-memory atom (row m's scale
 // of block kb at byte (m % 32) * 16 + (m / 32) * 4 + kb). Both operands'
 // scales are stored in that form in global memory, so a stage moves them
-// with one bulk copy each:
+// with one copy each:
 //  - activations, tile-blocked: for m-tile g (the 128-row tiles of all
-//    experts, numbered expert by expert) and stage q, 1 KB at (g * nst + q) *
-//    1024 (hi atom, then lo atom), written by the quantiser / mlp1's epilogue;
+//    experts, numbered expert by expert) and stage q, a 2 KB block at
+//    (g * nst + q) * 2048 (hi atom, lo atom, the small-expert kernel's atom),
+//    written by the quantiser / mlp1's epilogue;
 //  - weights, per (expert, column tile, stage): 1 KB (two atoms, rows 0..127
 //    and 128..255 of the tile), written from the (E, N, K/32) scales by a
-//    preparation pass before each GEMM (13 MB read at the 20B shape).
-// TMA's 4-bit type needs K to be a multiple of 128; for K % 128 = 64
-// (GPT-OSS: 2880) the same pass writes each weight row's last 64 codes
-// padded with zeros to a 128-element row, loaded by a second tensor map.
+//    preparation pass, per call for the experts a call routes to (13 MB read
+//    at the 20B shape) or once for all experts (moe_mxfp4_prepare).
+// The codes are read either as stored, (E, N, K/2) bytes (each stage a
+// 64-byte piece of every row, rows K/2 bytes apart; TMA's 4-bit type needs
+// K to be a multiple of 128, so for K % 128 = 64 (GPT-OSS: 2880) the per-call
+// pass writes each weight row's last 64 codes padded with zeros to a
+// 128-element row, loaded through a second tensor map), or from the
+// prepare-once copy, K-block-major (E, nst, N, 64 bytes) with the last block
+// padded, where a stage's rows are one contiguous run per half: 64-byte
+// pieces of rows 1.4 KB apart leave DRAM at about half its bandwidth.
 //
 // Every mbarrier wait is bounded (1 s); on timeout the kernel records
 // MOE_ERR_TIMEOUT, stops issuing, waits for its in-flight copies and MMAs,
@@ -71,7 +82,8 @@ using namespace sm100;
 constexpr int BM = 128;                                   // token rows per tile = TMEM lanes
 constexpr int BKE = 128;                                  // K elements per stage (4 scale blocks)
 constexpr int kStages = 3;
-constexpr int kThreads = 192;                             // producer, MMA, 4 epilogue warps
+constexpr int kThreads = 224;                             // 2 producers, MMA, 4 epilogue warps
+constexpr int kWProducerWarp = 6;                         // the weight-side producer
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;                      // accumulators at columns 0 and 256
 // Two 16-column scale-factor regions, used by alternate stages: after
@@ -87,8 +99,8 @@ struct MxParams {
   GemmParams g;            // sizes, bias, perm / gate weights, output, status, activation
   int nst;                 // 128-K stages
   int kfull;               // K rounded down to a multiple of 128 (the rest comes from the tail rows)
+  int wprep;               // codes from the prepared copy (K-block-major), else from the weights as stored
   const uint8_t* a_sf;     // activation scales, tile-blocked (nst stages)
-  const uint8_t* w_sf;     // weight scales: 1 KB per (expert, column tile, stage)
   uint8_t* hq;             // mlp1, optional: h quantised, hi (R, I) then lo (R, I) E4M3
   uint8_t* h_sf;           // and its scales, tile-blocked with h_nst stages
   int h_nst;
@@ -326,16 +338,23 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint16_t* __restric
 
 // ---------------------------------------------------------------- weight preparation
 // The weight scales in the atom layout the MMA's scale copies read, and the
-// ragged-K tail of the codes, for the experts each GEMM kernel takes:
+// codes in the form the GEMM kernels load, for the experts each kernel takes:
 //  - big-tile kernel (more than small_max rows): 1 KB per (expert, column
 //    tile, stage), two atoms for the tile's mma_n weight rows;
 //  - small-expert kernel (1..small_max rows): 512 B per (expert, weight tile,
 //    stage), one atom for its 128 weight rows (mlp1: 64 gate, 64 up);
-//  - with K % 128 = 64, each weight row's last 64 codes padded with zeros to a
-//    128-element row (64 bytes), for the 4-bit TMA type.
+//  - per call (codes read as stored, row by row): with K % 128 = 64, each
+//    weight row's last 64 codes padded with zeros to a 128-element row (64
+//    bytes), for the 4-bit TMA type;
+//  - prepare-once form: the codes K-block-major, (E, nst, N, 64 bytes), the
+//    128 codes of every row for K block q side by side and the ragged last
+//    block padded with zeros. A stage's weight rows are then one contiguous
+//    run per gate / up half (whole DRAM pages, where reading 64-byte pieces of
+//    rows K/2 bytes apart leaves DRAM at a fraction of its bandwidth).
 // With all_experts set (the prepare-once form) every expert gets both atom
-// sets and its tail rows; otherwise only what this call's routing uses.
-// One CTA per (expert, tile) or per 256 weight rows of an expert.
+// sets and its codes; otherwise only what this call's routing uses, and the
+// tail rows. One CTA per (expert, tile), per 256 weight rows of an expert, or
+// per (expert, K block, 64 weight rows).
 struct PrepArgs {
   const uint8_t* codes;
   const uint8_t* scales;
@@ -344,7 +363,8 @@ struct PrepArgs {
   int small_max, all_experts;
   uint8_t* w_sf;
   uint8_t* w_sf_small;
-  uint8_t* tail;
+  uint8_t* tail;       // per call with K % 128 != 0, else null
+  uint8_t* codes_out;  // prepare-once form, else null
 };
 
 __global__ void __launch_bounds__(256) mx_prep_weights_kernel(const PrepArgs a) {
@@ -352,6 +372,7 @@ __global__ void __launch_bounds__(256) mx_prep_weights_kernel(const PrepArgs a) 
   const int64_t wrows_all = static_cast<int64_t>(a.E) * a.b_rows;
   const int n_big = a.E * a.NT, n_small = a.small_max > 0 ? a.E * a.NT2 : 0;
   const int rblocks = (a.b_rows + 255) / 256;
+  const int n_tail = a.tail ? a.E * rblocks : 0;
   int blk = blockIdx.x;
   // the 4 scale bytes of a weight row for stage q (127 = 1.0 past K or past the tensor)
   auto sc4 = [&](int64_t row, int q) -> uint32_t {
@@ -391,9 +412,9 @@ __global__ void __launch_bounds__(256) mx_prep_weights_kernel(const PrepArgs a) 
     return;
   }
   blk -= n_small;
-  if (kfull < a.K) {
+  if (blk < n_tail) {
     const int e = blk / rblocks, rb = blk - e * rblocks;
-    if (e >= a.E || (!a.all_experts && count(e) <= 0)) return;
+    if (!a.all_experts && count(e) <= 0) return;
     for (int i = threadIdx.x; i < 256 * 4; i += blockDim.x) {
       const int r = rb * 256 + (i >> 2), piece = i & 3;
       if (r >= a.b_rows) break;
@@ -402,15 +423,31 @@ __global__ void __launch_bounds__(256) mx_prep_weights_kernel(const PrepArgs a) 
       if (piece < 2) v = __ldg(reinterpret_cast<const uint4*>(a.codes + row * half_k + kfull / 2 + piece * 16));
       *reinterpret_cast<uint4*>(a.tail + row * 64 + piece * 16) = v;
     }
+    return;
+  }
+  blk -= n_tail;
+  if (a.codes_out) {
+    // 64 rows of K block q of expert e, 16 bytes per thread
+    const int rchunks = (a.b_rows + 63) / 64;
+    const int e = blk / (a.nst * rchunks), rem = blk - e * (a.nst * rchunks);
+    const int q = rem / rchunks, rc = rem - q * rchunks;
+    if (e >= a.E) return;
+    const int r = rc * 64 + (threadIdx.x >> 2), piece = threadIdx.x & 3;
+    if (r >= a.b_rows) return;
+    const int64_t row = static_cast<int64_t>(e) * a.b_rows + r;
+    const int byte = q * 64 + piece * 16;  // within the stored row of K/2 bytes
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (byte < half_k) v = __ldg(reinterpret_cast<const uint4*>(a.codes + row * half_k + byte));
+    *reinterpret_cast<uint4*>(a.codes_out + ((static_cast<int64_t>(e) * a.nst + q) * a.b_rows + r) * 64 + piece * 16) = v;
   }
 }
 
 // ---------------------------------------------------------------- the block-scaled grouped GEMM
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1)
-    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmAhi, const __grid_constant__ CUtensorMap tmAlo,
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsf,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBtail,
-                   const MxParams p) {
+                   const __grid_constant__ CUtensorMap tmBsf, const MxParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const GemmParams& gp = p.g;
@@ -420,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = smem;
   uint8_t* ctrl = ring + kStages * sst;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
-  constexpr int kBars = 2 * kStages + 5;
+  constexpr int kBars = 3 * kStages + 5;
   static_assert(8 * kBars + 16 <= kCtrlBytes, "control block overflow");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -431,11 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
   const uint32_t bar0 = smem_u32(bars);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto tfull = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
-  auto tempty = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
-  const uint32_t done_bar = bar0 + 8u * (2 * kStages + 4);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };                // activation side landed
+  auto full_w = [&](int s) { return bar0 + 8u * (kStages + s); };      // weight side landed
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (3 * kStages + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (3 * kStages + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (3 * kStages + 4);
 
   // ---- prologue: segments, tile prefixes, barriers, TMEM
   if (warp == 0) {
@@ -451,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *total_s = ok ? tpre[gp.E] : 0;
       for (int s = 0; s < kStages; ++s) {
         mbar_init(full_bar(s), 1);
+        mbar_init(full_w(s), 1);
         mbar_init(empty_bar(s), 1);
       }
       for (int b = 0; b < 2; ++b) {
@@ -459,10 +498,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_init(done_bar, 1);
       fence_mbar_init();
-      tma_prefetch_desc(&tmAhi);
-      tma_prefetch_desc(&tmAlo);
-      if (p.kfull > 0) tma_prefetch_desc(&tmB);
-      if (p.kfull < gp.K) tma_prefetch_desc(&tmBtail);
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmAsf);
+      if (p.wprep || p.kfull > 0) tma_prefetch_desc(&tmB);
+      if (!p.wprep && p.kfull < gp.K) tma_prefetch_desc(&tmBtail);
+      tma_prefetch_desc(&tmBsf);
     }
   } else if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -480,10 +520,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nst = p.nst;
   const int nfull = p.kfull / BKE;  // stages whose codes come from the weights; the last, if ragged, from the tail rows
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kWProducerWarp) {
     if (lane == 0) {
-      // ---------------------------------------------------------- producer
-      const uint32_t stage_tx = kAStageBytes + static_cast<uint32_t>(gp.mma_n) * (BKE / 2) + 1024;
+      // ---------------------------------------------------------- producers
+      // A thread that issues a TMA copy waits ~60 ns before it can issue the
+      // next, whatever the copy's size, so a stage takes one copy per operand
+      // (hi and lo planes in one 3-D box; gate and up halves in one box) and
+      // two threads share them: warp 0 the activation side, warp 6 the weight
+      // side, each completing its own full barrier.
+      const bool wside = warp == kWProducerWarp;
+      const uint32_t stage_tx =
+          wside ? static_cast<uint32_t>(gp.mma_n) * (BKE / 2) + 1024 : 2 * kAOpBytes + 1024;
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool failed = false;
@@ -492,23 +539,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_tile(tile, tpre, seg, gp.E, BM, e, nt, mt);
         const int row0 = seg[e] + mt * BM;
         const int64_t g = mpre[e] + mt;
-        const int brow = e * gp.b_rows + nt * gp.n_tile;
-        const uint8_t* wsf = p.w_sf + (static_cast<int64_t>(e) * gp.NT + nt) * nst * 1024;
+        const int brow = nt * gp.n_tile;  // the tile's first (gate) row within the expert
+        const int64_t wsf_row = (static_cast<int64_t>(e) * gp.NT + nt) * nst;
         for (int q = 0; q < nst; ++q) {
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
             failed = true;
             break;
           }
           const uint32_t st = smem_u32(ring + s * sst);
-          mbar_arrive_expect_tx(full_bar(s), stage_tx);
-          tma_load_2d(st, &tmAhi, full_bar(s), q * BKE, row0);
-          tma_load_2d(st + kAOpBytes, &tmAlo, full_bar(s), q * BKE, row0);
-          bulk_load(st + 2 * kAOpBytes, p.a_sf + (g * nst + q) * kSfBlock, 1024, full_bar(s));
-          const CUtensorMap* tb = q < nfull ? &tmB : &tmBtail;
-          const int bx = q < nfull ? q * BKE : 0;
-          tma_load_2d(st + kBOff, tb, full_bar(s), bx, brow);
-          if (kSwiGLU) tma_load_2d(st + kBOff + gp.n_tile * 128, tb, full_bar(s), bx, brow + gp.n_out);
-          bulk_load(st + sfb_off, wsf + q * 1024, 1024, full_bar(s));
+          const uint32_t fb = wside ? full_w(s) : full_bar(s);
+          mbar_arrive_expect_tx(fb, stage_tx);
+          if (!wside) {
+            tma_load_3d(st, &tmA, fb, q * BKE, row0, 0);                                  // hi, lo planes
+            tma_load_2d(st + 2 * kAOpBytes, &tmAsf, fb, 0, static_cast<int32_t>(g * nst + q));  // their scales
+          } else {
+            if (p.wprep)
+              tma_load_4d(st + kBOff, &tmB, fb, 0, brow, 0, e * nst + q);
+            else if (q < nfull)
+              tma_load_4d(st + kBOff, &tmB, fb, q * BKE, e * gp.b_rows + brow, 0, 0);
+            else
+              tma_load_4d(st + kBOff, &tmBtail, fb, 0, e * gp.b_rows + brow, 0, 0);
+            tma_load_2d(st + sfb_off, &tmBsf, fb, 0, static_cast<int32_t>(wsf_row + q));
+          }
           ++issued;
           if (++s == kStages) {
             s = 0;
@@ -519,13 +571,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (failed) {
         record_status(gp.status, MOE_ERR_TIMEOUT);
         *abort_flag = 1;
-        const int n = issued < kStages ? issued : kStages;  // copies still in flight
+        const int n = issued < kStages ? issued : kStages;  // this thread's copies still in flight
         for (int i = 0; i < n; ++i) {
           if (--s < 0) {
             s = kStages - 1;
             ph ^= 1u;
           }
-          mbar_wait_bounded(full_bar(s), ph, nullptr, kWaitNs);
+          mbar_wait_bounded(wside ? full_w(s) : full_bar(s), ph, nullptr, kWaitNs);
         }
       }
     }
@@ -545,7 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kAccStride;
       for (int q = 0; q < nst; ++q) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs) &&
+                                         mbar_wait_bounded(full_w(s), ph, abort_flag, kWaitNs))) {
           failed = true;
           break;
         }
@@ -585,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_commit_elect(done_bar);
     mbar_wait_bounded(done_bar, 0, nullptr, kWaitNs);
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;  // TMEM lane quarter this warp may access
     const int m = qd * 32 + lane;
@@ -672,10 +725,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // its N side, hi rows over lo rows (N = 64), one MMA per 32-K block. Each tile
 // streams its weight rows once through a deep ring of small stages, so the
 // kernel runs at the rate HBM delivers the 4.25-bit weights.
-//   warp 0      producer, per stage: the weight codes (TMA 16U4_ALIGN16B),
-//               the expert's hi and lo rows (TMA, 32-row boxes), the weight
-//               rows' scale atom (bulk copy from the preparation pass) and the
-//               rows' 64-row scale atom (bulk copy from the activation scales);
+//   warp 0      weight-side producer, per stage: the weight codes (one TMA
+//               box, 16U4_ALIGN16B, both mlp1 halves) and the weight rows'
+//               scale atom (TMA, from the preparation pass);
+//   warp 6      row-side producer, per stage: the expert's hi and lo rows (one
+//               3-D TMA box of 32 rows x 2 planes) and their 64-row scale atom
+//               (TMA, from the activation scales);
 //   warps 1, 7  MMA: two scale copies into tensor memory and 4 block-scaled
 //               MMAs per stage; each warp takes alternate stages into its own
 //               accumulator (one warp alone issues a stage more slowly than HBM
@@ -700,19 +755,19 @@ constexpr uint32_t kSSfBase = 256;                   // scale regions (issuer i,
 constexpr int kSMaxStages = 8;
 constexpr int kXStride = 33;                         // floats per row of the up-half exchange buffer
 
-// Control block: 2 * stages + 9 mbarriers, then the TMEM slot, abort flag and
+// Control block: 3 * stages + 9 mbarriers, then the TMEM slot, abort flag and
 // tile total (16 bytes).
 __host__ __device__ constexpr uint32_t small_ctrl_bytes(int stages) {
-  return (8u * static_cast<uint32_t>(2 * stages + 9) + 16u + 15u) / 16u * 16u;
+  return (8u * static_cast<uint32_t>(3 * stages + 9) + 16u + 15u) / 16u * 16u;
 }
+constexpr int kSRowProducerWarp = 6;
 
 struct SmallParams {
   GemmParams g;           // E, K, n_out, b_rows, R, offsets, bias, perm, topk_w, out, status, act
   int nst, kfull;
   int NT2;                // weight tiles per expert
   int stages;             // ring depth
-  const uint8_t* w_sf;    // weight scale atoms: 512 B per (expert, weight tile, stage)
-  const uint8_t* a_sf;    // activation scales, tile-blocked
+  int wprep;              // codes from the prepared copy (K-block-major), else from the weights as stored
   uint8_t* hq;
   uint8_t* h_sf;
   int h_nst;
@@ -760,8 +815,8 @@ __device__ __forceinline__ void quant32_warp(float v, uint32_t& qh, uint32_t& ql
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kSThreads, 1)
     mx_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWtail,
-                    const __grid_constant__ CUtensorMap tmXhi, const __grid_constant__ CUtensorMap tmXlo,
-                    const SmallParams p) {
+                    const __grid_constant__ CUtensorMap tmWsf, const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmXsf, const SmallParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const GemmParams& gp = p.g;
@@ -770,7 +825,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
   float* xbuf = reinterpret_cast<float*>(ring + S * kSStage);  // 64 x kXStride
   uint8_t* ctrl = reinterpret_cast<uint8_t*>(xbuf + 64 * kXStride);
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
-  const int nbars = 2 * S + 9;
+  const int nbars = 3 * S + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * nbars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
@@ -780,12 +835,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
 
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
   const uint32_t bar0 = smem_u32(bars);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-  auto tfull = [&](int b) { return bar0 + 8u * (2 * S + b); };
-  auto tempty = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
-  const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
-  const uint32_t xfull = bar0 + 8u * (2 * S + 5), xempty = bar0 + 8u * (2 * S + 6);  // up-half exchange
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };            // weight side landed
+  auto full_x = [&](int s) { return bar0 + 8u * (S + s); };         // row side landed
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (3 * S + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (3 * S + 4);
+  const uint32_t xfull = bar0 + 8u * (3 * S + 5), xempty = bar0 + 8u * (3 * S + 6);  // up-half exchange
 
   if (warp == 0) {
     const bool ok = load_segments(gp.offsets, gp.E, gp.R, seg, mpre, gp.status);
@@ -796,6 +852,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       *total_s = ok ? tpre[gp.E] : 0;
       for (int s = 0; s < S; ++s) {
         mbar_init(full_bar(s), 1);
+        mbar_init(full_x(s), 1);
         mbar_init(empty_bar(s), 1);
       }
       for (int b = 0; b < 2; ++b) {
@@ -806,10 +863,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
       mbar_init(xfull, 2);
       mbar_init(xempty, 2);
       fence_mbar_init();
-      if (p.kfull > 0) tma_prefetch_desc(&tmW);
-      if (p.kfull < gp.K) tma_prefetch_desc(&tmWtail);
-      tma_prefetch_desc(&tmXhi);
-      tma_prefetch_desc(&tmXlo);
+      if (p.wprep || p.kfull > 0) tma_prefetch_desc(&tmW);
+      if (!p.wprep && p.kfull < gp.K) tma_prefetch_desc(&tmWtail);
+      tma_prefetch_desc(&tmWsf);
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmXsf);
     }
   } else if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -837,10 +895,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
     wt = tile - tpre[e];
   };
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kSRowProducerWarp) {
     if (lane == 0) {
-      // ---------------------------------------------------------- producer
-      constexpr uint32_t stage_tx = 128 * (BKE / 2) + kSB + 1024;
+      // ---------------------------------------------------------- producers
+      // (one TMA copy per operand per stage, two issuing threads: a thread
+      // waits ~60 ns after each copy it issues before the next)
+      const bool xside = warp == kSRowProducerWarp;
+      const uint32_t stage_tx = xside ? kSB + 512 : 128 * (BKE / 2) + 512;
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool failed = false;
@@ -849,23 +910,28 @@ __global__ void __launch_bounds__(kSThreads, 1)
         decode(tile, e, wt);
         const int row0 = seg[e];
         const int64_t g = mpre[e];
-        const int64_t wr = static_cast<int64_t>(e) * gp.b_rows + (kSwiGLU ? wt * 64 : wt * 128);
-        const uint8_t* wsf = p.w_sf + (static_cast<int64_t>(e) * p.NT2 + wt) * nst * 512;
+        const int wrow = kSwiGLU ? wt * 64 : wt * 128;  // the tile's first (gate) row within the expert
+        const int64_t wsf_row = (static_cast<int64_t>(e) * p.NT2 + wt) * nst;
         for (int q = 0; q < nst; ++q) {
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
             failed = true;
             break;
           }
           const uint32_t st = smem_u32(ring + s * kSStage);
-          mbar_arrive_expect_tx(full_bar(s), stage_tx);
-          const CUtensorMap* tw = q < nfull ? &tmW : &tmWtail;
-          const int wx = q < nfull ? q * BKE : 0;
-          tma_load_2d(st, tw, full_bar(s), wx, static_cast<int32_t>(wr));
-          if (kSwiGLU) tma_load_2d(st + 64 * 128, tw, full_bar(s), wx, static_cast<int32_t>(wr + gp.n_out));
-          tma_load_2d(st + kSA, &tmXhi, full_bar(s), q * BKE, row0);
-          tma_load_2d(st + kSA + kSmallRows * 128, &tmXlo, full_bar(s), q * BKE, row0);
-          bulk_load(st + kSA + kSB, wsf + q * 512, 512, full_bar(s));
-          bulk_load(st + kSA + kSB + 512, p.a_sf + (g * nst + q) * kSfBlock + 1024, 512, full_bar(s));
+          const uint32_t fb = xside ? full_x(s) : full_bar(s);
+          mbar_arrive_expect_tx(fb, stage_tx);
+          if (xside) {
+            tma_load_3d(st + kSA, &tmX, fb, q * BKE, row0, 0);  // hi rows over lo rows
+            tma_load_2d(st + kSA + kSB + 512, &tmXsf, fb, 0, static_cast<int32_t>(g * nst + q));
+          } else {
+            if (p.wprep)
+              tma_load_4d(st, &tmW, fb, 0, wrow, 0, e * nst + q);
+            else if (q < nfull)
+              tma_load_4d(st, &tmW, fb, q * BKE, e * gp.b_rows + wrow, 0, 0);
+            else
+              tma_load_4d(st, &tmWtail, fb, 0, e * gp.b_rows + wrow, 0, 0);
+            tma_load_2d(st + kSA + kSB, &tmWsf, fb, 0, static_cast<int32_t>(wsf_row + q));
+          }
           ++issued;
           if (++s == S) {
             s = 0;
@@ -876,13 +942,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
       if (failed) {
         record_status(gp.status, MOE_ERR_TIMEOUT);
         *abort_flag = 1;
-        const int n = issued < S ? issued : S;  // copies still in flight
+        const int n = issued < S ? issued : S;  // this thread's copies still in flight
         for (int i = 0; i < n; ++i) {
           if (--s < 0) {
             s = S - 1;
             ph ^= 1u;
           }
-          mbar_wait_bounded(full_bar(s), ph, nullptr, kWaitNs);
+          mbar_wait_bounded(xside ? full_x(s) : full_bar(s), ph, nullptr, kWaitNs);
         }
       }
     }
@@ -904,7 +970,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
       const uint32_t d_tmem = tmem_base + (2 * iss + acc) * kSAccStride;
       for (int q = 0; q < nst; ++q) {
         if ((q & 1) == iss) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs))) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs) &&
+                                           mbar_wait_bounded(full_x(s), ph, abort_flag, kWaitNs))) {
             failed = true;
             break;
           }
@@ -1066,35 +1133,59 @@ __global__ void __launch_bounds__(kSThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-// (rows, inner) bytes, loaded as 128-byte x box_rows boxes with the 128-byte
-// swizzle (the K-major E4M3 operand layout).
-bool make_tmap_e4m3(CUtensorMap* map, const uint8_t* base, uint64_t inner, uint64_t rows, uint32_t box_rows = BM) {
+// Tensor maps (cuTensorMapEncodeTiled through the runtime's driver entry
+// point); a false return becomes MOE_ERR_CUDA.
+
+// The hi and lo E4M3 planes, (R, K) bytes each with lo right after hi, as one
+// 3-D tensor (K, R, 2) loaded in 128-byte x box_rows x 2 boxes with the
+// 128-byte swizzle: a stage's hi rows, then its lo rows, in shared memory.
+bool make_tmap_act(CUtensorMap* map, const uint8_t* hi, uint64_t K, uint64_t R, uint32_t box_rows) {
   auto fn = tma_encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+  cuuint64_t dims[3] = {K, R, 2};
+  cuuint64_t strides[2] = {K, R * K};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(BKE), box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(hi), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E2M1 codes of `rows` rows of row_bytes bytes: the first kfull elements of
-// each row (kfull a multiple of 128) as 128-element x box_rows boxes,
-// unpacked by TMA into the MMA's E2M1 operand layout (every 8 bytes of codes
-// padded to 16) with the 128-byte swizzle. The base must be 32-byte aligned
-// and row_bytes a multiple of 32.
-bool make_tmap_e2m1(CUtensorMap* map, const uint8_t* codes, uint64_t kfull, uint64_t row_bytes, uint64_t rows,
-                    uint32_t box_rows) {
+// E2M1 codes as a 4-D tensor (elements, rows, halves, K blocks): `inner`
+// elements per row (a multiple of 128), rows `row_bytes` apart, `halves` (2:
+// mlp1's gate rows and the matching up rows) `half_bytes` apart, `kblocks`
+// blocks `kblock_bytes` apart. Loaded as 128-element x box_rows x halves x 1
+// boxes, unpacked by TMA into the MMA's E2M1 operand layout (every 8 bytes of
+// codes padded to 16) with the 128-byte swizzle: the gate rows, then the up
+// rows, in shared memory. Base 32-byte aligned, strides multiples of 32.
+//  - weights as stored: (K rounded down to 128, E * N, halves, 1), rows K/2 bytes apart;
+//  - their tail rows: (128, E * N, halves, 1), rows 64 bytes apart;
+//  - the prepared copy: (128, rows per half, halves, E * nst), rows 64 bytes apart.
+bool make_tmap_codes(CUtensorMap* map, const uint8_t* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                     uint32_t halves, uint64_t half_bytes, uint64_t kblocks, uint64_t kblock_bytes,
+                     uint32_t box_rows) {
   auto fn = tma_encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {kfull, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKE), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+  cuuint64_t dims[4] = {inner, rows, halves, kblocks};
+  cuuint64_t strides[3] = {row_bytes, half_bytes, kblock_bytes};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(BKE), box_rows, halves, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// `count` scale atoms of atom_bytes (512 or 1024) bytes, `stride` bytes
+// apart, one atom per load, copied as is.
+bool make_tmap_atoms(CUtensorMap* map, const uint8_t* base, uint32_t atom_bytes, uint64_t count, uint64_t stride) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {atom_bytes / 4u, count};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {atom_bytes / 4u, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1121,23 +1212,24 @@ size_t small_smem_bytes(int stages, int E) {
          3 * static_cast<size_t>(E + 1) * sizeof(int);
 }
 
-// The preparation region of one GEMM: big-tile atoms, small-tile atoms, tail rows.
+// The preparation region of one GEMM: big-tile atoms, small-tile atoms, then
+// either (per call) the tail rows or (prepare-once form) the K-block-major codes.
 struct PrepLayout {
-  size_t big, small, tail, total;
+  size_t big, small, rest, tail, codes;
+  size_t per_call() const { return rest + tail; }
+  size_t prepared() const { return rest + codes; }
 };
 PrepLayout prep_layout(int E, int b_rows, int K, int NT, int NT2) {
   PrepLayout L{};
   const int nst = (K + BKE - 1) / BKE;
   L.big = 0;
   L.small = align_up(static_cast<size_t>(E) * NT * nst * 1024, 256);
-  L.tail = L.small + align_up(static_cast<size_t>(E) * NT2 * nst * 512, 256);
-  L.total = L.tail + (K % BKE ? align_up(static_cast<size_t>(E) * b_rows * 64, 256) : 0);
+  L.rest = L.small + align_up(static_cast<size_t>(E) * NT2 * nst * 512, 256);
+  L.tail = K % BKE ? align_up(static_cast<size_t>(E) * b_rows * 64, 256) : 0;
+  L.codes = align_up(static_cast<size_t>(E) * nst * b_rows * 64, 256);
   return L;
 }
 
-// One grouped GEMM with MXFP4 weights: the preparation pass, then the
-// small-expert kernel (experts with 1..kSmallRows rows) and the big-tile
-// kernel (the others), each skipping the other's experts.
 // The small-expert kernel's geometry for a GEMM: weight tiles per expert,
 // ring depth, and whether it runs at all (else every expert takes big tiles).
 struct SmallGeom {
@@ -1162,59 +1254,76 @@ moe_status_t run_prep(const MxParams& p, const uint8_t* codes, const uint8_t* sc
   const GemmParams& g = p.g;
   const SmallGeom sg = small_geom<kSwiGLU>(g);
   const PrepLayout L = prep_layout(g.E, g.b_rows, g.K, g.NT, sg.NT2);
+  uint8_t* tail = (!all_experts && g.K % BKE) ? out + L.rest : nullptr;
+  uint8_t* codes_out = all_experts ? out + L.rest : nullptr;
   PrepArgs pa{codes, scales, g.E, g.b_rows, g.K, g.n_out, g.n_tile, g.mma_n, g.NT, sg.NT2, p.nst, kSwiGLU ? 1 : 0,
-              g.offsets, sg.ok ? kSmallRows : 0, all_experts ? 1 : 0, out + L.big, out + L.small, out + L.tail};
-  const int blocks = g.E * g.NT + (sg.ok ? g.E * sg.NT2 : 0) + (g.K % BKE ? g.E * ((g.b_rows + 255) / 256) : 0);
-  mx_prep_weights_kernel<<<blocks, 256, 0, s>>>(pa);
+              g.offsets, sg.ok ? kSmallRows : 0, all_experts ? 1 : 0, out + L.big, out + L.small, tail, codes_out};
+  const int64_t blocks = static_cast<int64_t>(g.E) * g.NT + (sg.ok ? static_cast<int64_t>(g.E) * sg.NT2 : 0) +
+                         (tail ? static_cast<int64_t>(g.E) * ((g.b_rows + 255) / 256) : 0) +
+                         (codes_out ? static_cast<int64_t>(g.E) * p.nst * ((g.b_rows + 63) / 64) : 0);
+  if (blocks > 0x7fffffff) return MOE_ERR_UNSUPPORTED;
+  mx_prep_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(pa);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 template <bool kSwiGLU>
-size_t prep_bytes(const MxParams& p) {
-  return prep_layout(p.g.E, p.g.b_rows, p.g.K, p.g.NT, small_geom<kSwiGLU>(p.g).NT2).total;
+PrepLayout layout_of(const MxParams& p) {
+  return prep_layout(p.g.E, p.g.b_rows, p.g.K, p.g.NT, small_geom<kSwiGLU>(p.g).NT2);
 }
 
-// prep: the preparation region, written here per call (only what this call's
-// routing uses) unless `prepared` says it already holds the prepare-once form.
+// One grouped GEMM with MXFP4 weights: the preparation pass (unless `prep`
+// already holds the prepare-once form), then the small-expert kernel (experts
+// with 1..kSmallRows rows) and the big-tile kernel (the others), each
+// skipping the other's experts.
 template <bool kSwiGLU>
 moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8_t* scales, uint8_t* prep,
                             bool prepared, MxParams p, cudaStream_t s) {
   const GemmParams& g = p.g;
   p.kfull = g.K / BKE * BKE;
+  p.wprep = prepared ? 1 : 0;
   const SmallGeom sg = small_geom<kSwiGLU>(g);
-  SmallParams sp{};
-  sp.g = g;
-  sp.nst = p.nst;
-  sp.kfull = p.kfull;
-  sp.NT2 = sg.NT2;
-  sp.stages = sg.stages;
-  const bool small_ok = sg.ok;
-  p.small_max = small_ok ? kSmallRows : 0;
-  const PrepLayout L = prep_layout(g.E, g.b_rows, g.K, g.NT, sp.NT2);
-  uint8_t* w_sf = prep + L.big;
-  uint8_t* w_sf_small = prep + L.small;
-  uint8_t* tail = prep + L.tail;
+  const PrepLayout L = prep_layout(g.E, g.b_rows, g.K, g.NT, sg.NT2);
   if (!prepared) {
     const moe_status_t st = run_prep<kSwiGLU>(p, codes, scales, prep, false, s);
     if (st != MOE_OK) return st;
   }
-  p.w_sf = w_sf;
-  sp.w_sf = w_sf_small;
-  sp.a_sf = p.a_sf;
-  sp.hq = p.hq;
-  sp.h_sf = p.h_sf;
-  sp.h_nst = p.h_nst;
+  const int nst = p.nst;
   const uint64_t wrows = static_cast<uint64_t>(g.E) * g.b_rows;
-  const uint8_t* alo = aq + g.R * g.K;
+  const uint64_t row_bytes = static_cast<uint64_t>(g.K) / 2;
+  const uint32_t halves = kSwiGLU ? 2 : 1;
+  const uint64_t m_tiles = static_cast<uint64_t>((g.R + BM - 1) / BM + g.E);  // what the activation scales hold
+  // the weight codes (and, per call with a ragged K, the tail rows) in boxes of box_rows rows per half
+  auto codes_maps = [&](CUtensorMap* m, CUtensorMap* t, uint32_t box_rows) -> bool {
+    memset(m, 0, sizeof(*m));
+    memset(t, 0, sizeof(*t));
+    if (prepared)
+      return make_tmap_codes(m, prep + L.rest, BKE, g.n_out, 64, halves, static_cast<uint64_t>(g.n_out) * 64,
+                             static_cast<uint64_t>(g.E) * nst, static_cast<uint64_t>(g.b_rows) * 64, box_rows);
+    if (p.kfull > 0 && !make_tmap_codes(m, codes, p.kfull, wrows, row_bytes, halves, g.n_out * row_bytes, 1,
+                                        wrows * row_bytes, box_rows))
+      return false;
+    if (p.kfull < g.K && !make_tmap_codes(t, prep + L.rest, BKE, wrows, 64, halves, static_cast<uint64_t>(g.n_out) * 64,
+                                          1, wrows * 64, box_rows))
+      return false;
+    return true;
+  };
 
-  if (small_ok) {
-    CUtensorMap tw, twt, txh, txl;
-    memset(&tw, 0, sizeof(tw));
-    memset(&twt, 0, sizeof(twt));
-    const uint32_t wbox = kSwiGLU ? 64 : 128;
-    if (p.kfull > 0 && !make_tmap_e2m1(&tw, codes, p.kfull, g.K / 2, wrows, wbox)) return MOE_ERR_CUDA;
-    if (p.kfull < g.K && !make_tmap_e2m1(&twt, tail, BKE, 64, wrows, wbox)) return MOE_ERR_CUDA;
-    if (!make_tmap_e4m3(&txh, aq, g.K, g.R, kSmallRows) || !make_tmap_e4m3(&txl, alo, g.K, g.R, kSmallRows))
+  if (sg.ok) {
+    SmallParams sp{};
+    sp.g = g;
+    sp.nst = nst;
+    sp.kfull = p.kfull;
+    sp.NT2 = sg.NT2;
+    sp.stages = sg.stages;
+    sp.wprep = p.wprep;
+    sp.hq = p.hq;
+    sp.h_sf = p.h_sf;
+    sp.h_nst = p.h_nst;
+    CUtensorMap tw, twt, twsf, tx, txsf;
+    if (!codes_maps(&tw, &twt, kSwiGLU ? 64 : 128) ||
+        !make_tmap_atoms(&twsf, prep + L.small, 512, static_cast<uint64_t>(g.E) * sg.NT2 * nst, 512) ||
+        !make_tmap_act(&tx, aq, g.K, g.R, kSmallRows) ||
+        !make_tmap_atoms(&txsf, p.a_sf + 1024, 512, m_tiles * nst, kSfBlock))
       return MOE_ERR_CUDA;
     const size_t smem = small_smem_bytes(sp.stages, g.E);
     if (cudaFuncSetAttribute(mx_small_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1222,17 +1331,16 @@ moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8
       return MOE_ERR_CUDA;
     const int64_t max_tiles = static_cast<int64_t>(g.E) * sp.NT2;
     const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-    mx_small_kernel<kSwiGLU><<<grid, kSThreads, smem, s>>>(tw, twt, txh, txl, sp);
+    mx_small_kernel<kSwiGLU><<<grid, kSThreads, smem, s>>>(tw, twt, twsf, tx, txsf, sp);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
+  p.small_max = sg.ok ? kSmallRows : 0;
 
-  CUtensorMap thi, tlo, tb, tt;
-  memset(&tb, 0, sizeof(tb));
-  memset(&tt, 0, sizeof(tt));
-  if (!make_tmap_e4m3(&thi, aq, g.K, g.R) || !make_tmap_e4m3(&tlo, alo, g.K, g.R)) return MOE_ERR_CUDA;
-  const uint32_t box_rows = static_cast<uint32_t>(kSwiGLU ? g.n_tile : g.mma_n);
-  if (p.kfull > 0 && !make_tmap_e2m1(&tb, codes, p.kfull, g.K / 2, wrows, box_rows)) return MOE_ERR_CUDA;
-  if (p.kfull < g.K && !make_tmap_e2m1(&tt, tail, BKE, 64, wrows, box_rows)) return MOE_ERR_CUDA;
+  CUtensorMap ta, tasf, tb, tt, tbsf;
+  if (!make_tmap_act(&ta, aq, g.K, g.R, BM) || !make_tmap_atoms(&tasf, p.a_sf, 1024, m_tiles * nst, kSfBlock) ||
+      !codes_maps(&tb, &tt, static_cast<uint32_t>(kSwiGLU ? g.n_tile : g.mma_n)) ||
+      !make_tmap_atoms(&tbsf, prep + L.big, 1024, static_cast<uint64_t>(g.E) * g.NT * nst, 1024))
+    return MOE_ERR_CUDA;
   const size_t smem = smem_bytes(g.mma_n, g.E);
   if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(mx_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1240,7 +1348,7 @@ moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8
     return MOE_ERR_CUDA;
   const int64_t max_tiles = ((g.R + BM - 1) / BM + g.E) * static_cast<int64_t>(g.NT);
   const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  mx_gemm_kernel<kSwiGLU><<<grid, kThreads, smem, s>>>(thi, tlo, tb, tt, p);
+  mx_gemm_kernel<kSwiGLU><<<grid, kThreads, smem, s>>>(ta, tasf, tb, tt, tbsf, p);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -1249,12 +1357,6 @@ moe_status_t launch_mx_gemm(const uint8_t* aq, const uint8_t* codes, const uint8
 size_t mx_sf_bytes(const moe_dims_t& d, int K) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
   return static_cast<size_t>((R + BM - 1) / BM + d.E) * ((K + BKE - 1) / BKE) * kSfBlock;
-}
-
-size_t mx_prep_bytes(const moe_dims_t& d) {
-  const size_t p1 = mx_prepared_bytes(d, 1), p2 = mx_prepared_bytes(d, 2);
-  if (p1 == 0 || p2 == 0) return 0;
-  return align_up(p1 > p2 ? p1 : p2, 256);
 }
 
 moe_status_t launch_mx_quant(const moe_dims_t& d, const uint16_t* src, const int32_t* perm, int K,
@@ -1335,13 +1437,20 @@ moe_status_t launch_mlp2_mx(const moe_dims_t& d, const uint8_t* hq, const uint8_
 size_t mx_prepared_bytes(const moe_dims_t& d, int which) {
   if (which == 1) {
     const MxParams p = mlp1_params(d);
-    return p.g.n_tile ? prep_bytes<true>(p) : 0;
+    return p.g.n_tile ? layout_of<true>(p).prepared() : 0;
   }
   if (which == 2) {
     const MxParams p = mlp2_params(d);
-    return p.g.n_tile ? prep_bytes<false>(p) : 0;
+    return p.g.n_tile ? layout_of<false>(p).prepared() : 0;
   }
   return 0;
+}
+
+size_t mx_prep_bytes(const moe_dims_t& d) {
+  const MxParams p1 = mlp1_params(d), p2 = mlp2_params(d);
+  if (p1.g.n_tile == 0 || p2.g.n_tile == 0) return 0;
+  const size_t b1 = layout_of<true>(p1).per_call(), b2 = layout_of<false>(p2).per_call();
+  return align_up(b1 > b2 ? b1 : b2, 256);
 }
 
 moe_status_t mx_prepare(const moe_dims_t& d, int which, const uint8_t* codes, const uint8_t* scales, uint8_t* out,

@@ -175,11 +175,13 @@ def test_mxfp4_prepare_arguments():
     dq = moe.dims(64, 2880, 32, 4, 2880, wfmt=moe.MOE_W_MXFP4)
     n1, n2 = moe.mxfp4_prepared_bytes(dq, 1), moe.mxfp4_prepared_bytes(dq, 2)
     nst = -(-2880 // 128)
-    assert n1 >= 32 * 30 * nst * 1024 + 32 * 45 * nst * 512 + 32 * 5760 * 64
-    assert n2 >= 32 * 12 * nst * 1024 + 32 * 23 * nst * 512 + 32 * 2880 * 64
+    # scale atoms of both kernels, then the codes K-block-major (every block of
+    # 128 K padded to 64 bytes per row)
+    assert n1 >= 32 * 30 * nst * 1024 + 32 * 45 * nst * 512 + 32 * nst * 5760 * 64
+    assert n2 >= 32 * 12 * nst * 1024 + 32 * 23 * nst * 512 + 32 * nst * 2880 * 64
     assert moe.mxfp4_prepared_bytes(moe.dims(64, 2880, 32, 4, 2880), 1) == 0  # bf16 weights
     assert moe.mxfp4_prepared_bytes(dq, 3) == 0
-    ar = _Arena(96 << 20)
+    ar = _Arena(n1 + (64 << 20))
     vp = ctypes.c_void_p
     w = _binding.Weight(ar.take(), ar.take(), None)
     out = vp(ar.take(n1))

@@ -139,9 +139,9 @@ def test_mxfp4_prepared_weights_match_per_call(T, D, E, k, I):
     assert moe.moe_read_device_status(ws) == 0
     assert torch.equal(h.view(torch.int16), run.h.view(torch.int16))
     assert torch.equal(o, run.o_perm)
+    # with the prepared forms the GEMMs read nothing else: codes and scales omitted
     y = torch.empty((s.T, s.D), dtype=BF16, device="cuda")
-    moe.moe_forward(d, inp.x, inp.Wr, inp.br, inp.W1, inp.b1, inp.W2, inp.b2, y, ws, W1_scales=inp.W1_scales,
-                    W2_scales=inp.W2_scales, W1_prepared=p1, W2_prepared=p2)
+    moe.moe_forward(d, inp.x, inp.Wr, inp.br, None, inp.b1, None, inp.b2, y, ws, W1_prepared=p1, W2_prepared=p2)
     assert moe.moe_read_device_status(ws) == 0
     assert torch.equal(y.view(torch.int16), run.y.view(torch.int16))
 
