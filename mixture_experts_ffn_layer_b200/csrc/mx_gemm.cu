@@ -731,11 +731,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warp 6      row-side producer, per stage: the expert's hi and lo rows (one
 //               3-D TMA box of 32 rows x 2 planes) and their 64-row scale atom
 //               (TMA, from the activation scales);
-//   warps 1, 7  MMA: two scale copies into tensor memory and 4 block-scaled
-//               MMAs per stage; each warp takes alternate stages into its own
-//               accumulator (one warp alone issues a stage more slowly than HBM
-//               delivers it);
-//   warps 2..5  epilogue (lane = weight row): both issuers' hi + lo parts
+//   warps 1,7,8 MMA: two scale copies into tensor memory and 4 block-scaled
+//               MMAs per stage; warp i takes the stages q = i mod 3 into its
+//               own accumulator. Each tcgen05 instruction holds its issuing
+//               warp for ~50 ns, so one warp needs ~0.4 us per stage where HBM
+//               delivers one in ~0.2; issuing from three warps overlaps it;
+//   warps 2..5  epilogue (lane = weight row): the issuers' hi + lo parts
 //               added per row in a fixed order, then SwiGLU with the up half
 //               from the other two warps via shared memory and h quantised
 //               across the warp's 32 columns, or bias * gate weight into the
@@ -744,14 +745,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // copies, so no proxy fence sits on the pipeline.
 constexpr int kSmallRows = 32;
 constexpr int kSN = 2 * kSmallRows;                  // the expert's hi rows, then its lo rows
-constexpr int kSThreads = 256;
-constexpr int kSIssuers = 2;
-constexpr int kSMma1Warp = 7;
+constexpr int kSThreads = 288;
+constexpr int kSIssuers = 3;
+__device__ __forceinline__ int small_issuer_of(int warp) { return warp == 1 ? 0 : warp == 7 ? 1 : warp == 8 ? 2 : -1; }
 constexpr uint32_t kSA = 128 * 128;                  // weight operand: 128 rows x 128 B
 constexpr uint32_t kSB = kSN * 128;                  // row operand: 64 rows x 128 B
 constexpr uint32_t kSStage = kSA + kSB + 1024;       // + weight scale atom, row scale atom (512 B each)
 constexpr uint32_t kSAccStride = 64;                 // accumulator (issuer i, buffer b) at (2i + b) * 64
-constexpr uint32_t kSSfBase = 256;                   // scale regions (issuer i, r) at 256 + (2i + r) * 8
+constexpr uint32_t kSSfBase = 384;                   // scale regions (issuer i, r) at 384 + (2i + r) * 8
+static_assert(kSSfBase >= 2 * kSIssuers * kSAccStride && kSSfBase + 16 * kSIssuers <= 512, "TMEM columns");
 constexpr int kSMaxStages = 8;
 constexpr int kXStride = 33;                         // floats per row of the up-half exchange buffer
 
@@ -952,11 +954,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == kSMma1Warp) {
+  } else if (small_issuer_of(warp) >= 0) {
     // ------------------------------------------------------------ MMA issuers (whole warp, one lane elected)
-    // Issuer i takes the stages q = i, i + 2, ... of every tile; both track
+    // Issuer i takes the stages q = i, i + 3, ... of every tile; all track
     // the ring position of every stage.
-    const int iss = warp == 1 ? 0 : 1;
+    const int iss = small_issuer_of(warp);
     const uint32_t idesc = idesc_mx(5 /* E2M1 weights */, 0 /* E4M3 rows */, kSN);
     int s = 0, acc = 0, sfr = 0;
     uint32_t ph = 0, pacc = 0;
@@ -969,7 +971,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (2 * iss + acc) * kSAccStride;
       for (int q = 0; q < nst; ++q) {
-        if ((q & 1) == iss) {
+        if (q % kSIssuers == iss) {
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs) &&
                                            mbar_wait_bounded(full_x(s), ph, abort_flag, kWaitNs))) {
             failed = true;
@@ -995,7 +997,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         }
       }
       if (failed) break;
-      tc_commit_elect(tfull(acc));  // issuer 1 with no stage (one-stage K) arrives at once
+      tc_commit_elect(tfull(acc));  // an issuer with no stage in the tile (short K) arrives at once
       if (++acc == 2) {
         acc = 0;
         pacc ^= 1u;
@@ -1027,8 +1029,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kSAccStride;
-      // row t's value: issuer 0's (hi + lo) part, plus issuer 1's when the
-      // tile had a second stage, added in that order
+      // row t's value: issuer 0's (hi + lo) part, then those of the issuers
+      // that had stages in this tile (issuer i when nst > i), added in that order
       float v[kSmallRows];
       {
         uint32_t hv[32], lv[32];
@@ -1037,9 +1039,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int t = 0; t < kSmallRows; ++t) v[t] = __uint_as_float(hv[t]) + __uint_as_float(lv[t]);
-        if (nst > 1) {
-          tmem_ld_x32(tb + 2 * kSAccStride, hv);
-          tmem_ld_x32(tb + 2 * kSAccStride + kSmallRows, lv);
+        for (int i = 1; i < kSIssuers && i < nst; ++i) {
+          tmem_ld_x32(tb + 2 * i * kSAccStride, hv);
+          tmem_ld_x32(tb + 2 * i * kSAccStride + kSmallRows, lv);
           tmem_ld_wait();
 #pragma unroll
           for (int t = 0; t < kSmallRows; ++t) v[t] += __uint_as_float(hv[t]) + __uint_as_float(lv[t]);
