@@ -133,20 +133,34 @@ class Clocks:
 
 
 GEMM_SOURCES = ("grouped_gemm.cu", "gemm_common.cuh", "sm100.cuh")
+MX_SOURCES = ("mx_gemm.cu", "gemm_common.cuh", "sm100.cuh", "common.cuh", "tma_host.cuh")
+# workload -> the ncu summary of its mlp1 kernel and the sources that kernel is built from
+PROFILE_OF = {
+    "gptoss20b": ("mlp1_gptoss20b_ncu.md", GEMM_SOURCES),
+    "gptoss20b_mxfp4": ("mx_gemm_gptoss20b_mxfp4_ncu.md", MX_SOURCES),
+    "gptoss20b_mxfp4_decode": ("mx_small_gptoss20b_mxfp4_decode_ncu.md", MX_SOURCES),
+}
 
 
-def gemm_source_hash() -> str:
-    """Hash of the sources that make up the mlp1 kernel."""
+def source_hash(sources=GEMM_SOURCES) -> str:
+    """Hash of the sources that make up a kernel."""
     h = hashlib.sha256()
-    for name in GEMM_SOURCES:
+    for name in sources:
         h.update(open(os.path.join(ROOT, "mixture_experts_ffn_layer_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile():
-    """DRAM bytes per launch of the mlp1 kernel from the committed ncu summary,
-    if it was taken on the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "mlp1_gptoss20b_ncu.md")
+def gemm_source_hash() -> str:
+    return source_hash(GEMM_SOURCES)
+
+
+def traffic_from_profile(workload=WORKLOAD):
+    """DRAM bytes per launch of the workload's mlp1 kernel from its committed
+    ncu summary, if that was taken on the current kernel sources; else None."""
+    if workload not in PROFILE_OF:
+        return None
+    name, sources = PROFILE_OF[workload]
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     fields = {}
@@ -154,7 +168,7 @@ def traffic_from_profile():
         m = re.match(r"- (\w+): `([^`]*)`", line)
         if m:
             fields[m.group(1)] = m.group(2)
-    if fields.get("kernel_sources_sha256_16") != gemm_source_hash():
+    if fields.get("kernel_sources_sha256_16") != source_hash(sources):
         return None
     try:
         return int(float(fields["dram_bytes_per_launch"]))
@@ -199,12 +213,13 @@ def rooflines(shape, inp, stage_ms, mlp1_ms, peak_tf, pk, pk_kind, workload):
         mlp1_bytes = w1_bytes + R * D * 2 + R * I * 2
         ach = mlp1_bytes / (mlp1_ms / 1e3) / 1e9
         roof = {"kernel": "grouped mlp1 + SwiGLU (tcgen05)", "bound": "hbm", "achieved": ach, "peak": hbm,
-                "unit": "GB/s", "frac": ach / hbm, "traffic": None, "peak_kind": f"hbm_gbs ({pk_kind})",
+                "unit": "GB/s", "frac": ach / hbm, "traffic": traffic_from_profile(workload),
+                "peak_kind": f"hbm_gbs ({pk_kind})",
                 "algorithmic": f"W1 {w1_bytes} B + routed rows {R * D * 2} B + h {R * I * 2} B per launch"}
     else:
         mlp1_flops = 4.0 * R * D * I
         tf = mlp1_flops / (mlp1_ms / 1e3) / 1e12
-        traffic = traffic_from_profile() if workload == WORKLOAD else None
+        traffic = traffic_from_profile(workload)
         roof = {"kernel": "grouped mlp1 + SwiGLU (tcgen05)", "bound": "tensor", "achieved": tf, "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": traffic,
                 "algorithmic": f"4*R*D*I = {mlp1_flops:.4g} FLOP per launch"}

@@ -487,6 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       *abort_flag = 0;
       *total_s = ok ? tpre[gp.E] : 0;
+    }
+  }
+  __syncthreads();
+  // A CTA without a tile (on decode-sized batches every expert may go to the
+  // small-expert kernel) leaves before it allocates tensor memory.
+  if (static_cast<int>(blockIdx.x) >= *total_s) return;
+  if (warp == 0) {
+    if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
         mbar_init(full_bar(s), 1);
         mbar_init(full_w(s), 1);
@@ -852,6 +860,14 @@ __global__ void __launch_bounds__(kSThreads, 1)
     if (lane == 0) {
       *abort_flag = 0;
       *total_s = ok ? tpre[gp.E] : 0;
+    }
+  }
+  __syncthreads();
+  // A CTA without a tile (on large batches no expert may have 1..32 rows)
+  // leaves before it allocates tensor memory.
+  if (static_cast<int>(blockIdx.x) >= *total_s) return;
+  if (warp == 0) {
+    if (lane == 0) {
       for (int s = 0; s < S; ++s) {
         mbar_init(full_bar(s), 1);
         mbar_init(full_x(s), 1);

@@ -50,21 +50,23 @@ def test_single_rank_is_identity():
     assert ms == 100.0 and value == pytest.approx(81920.0)
 
 
-def test_profile_traffic_is_read_for_the_profiled_kernel_sources(tmp_path, monkeypatch):
-    # the committed ncu summary carries the hash of the GEMM sources it was
+@pytest.mark.parametrize("workload", ["gptoss20b", "gptoss20b_mxfp4", "gptoss20b_mxfp4_decode"])
+def test_profile_traffic_is_read_for_the_profiled_kernel_sources(tmp_path, monkeypatch, workload):
+    # each committed ncu summary carries the hash of the kernel sources it was
     # taken on; the bench reports its DRAM bytes only while that hash matches
-    p = os.path.join(bench.ROOT, "profiles", "mlp1_gptoss20b_ncu.md")
-    text = open(p).read()
+    name, sources = bench.PROFILE_OF[workload]
+    text = open(os.path.join(bench.ROOT, "profiles", name)).read()
     fake = tmp_path / "profiles"
     fake.mkdir()
-    (fake / "mlp1_gptoss20b_ncu.md").write_text(text)
+    (fake / name).write_text(text)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     import re
 
     sha = re.search(r"kernel_sources_sha256_16: `([0-9a-f]{16})`", text).group(1)
     nbytes = int(re.search(r"dram_bytes_per_launch: `(\d+)`", text).group(1))
-    monkeypatch.setattr(bench, "gemm_source_hash", lambda: sha)
-    assert bench.traffic_from_profile() == nbytes
+    monkeypatch.setattr(bench, "source_hash", lambda srcs: sha if srcs == sources else "0" * 16)
+    assert bench.traffic_from_profile(workload) == nbytes
     # a summary taken on other kernel sources is ignored
-    monkeypatch.setattr(bench, "gemm_source_hash", lambda: "f" * 16)
-    assert bench.traffic_from_profile() is None
+    monkeypatch.setattr(bench, "source_hash", lambda srcs: "f" * 16)
+    assert bench.traffic_from_profile(workload) is None
+    assert bench.traffic_from_profile("gptoss120b_zipf") is None  # no summary for this workload
