@@ -154,12 +154,13 @@ MOE_API moe_status_t moe_gather(moe_dims_t d, const uint16_t* x, const int32_t* 
  *   with act = d.act (plain SwiGLU or the GPT-OSS variant, see moe_act_t).
  *   x_perm (R,D) bf16, offsets (E+1), W1 (E,2I,D), b1 (E,2I) bf16 -> h (R,I) bf16.
  * tcgen05 tensor-core grouped GEMM, persistent over (expert, row tile, column tile).
- * MXFP4 weights: with T*k <= 16*E (a few rows per expert) the codes are
- * streamed once and decoded on chip into tcgen05 operands (weight-streaming
- * kernel, which takes the routed rows in f16: |x| must stay below 65504 and
- * |h| below 2^24 there, far above what a layer's activations reach);
- * otherwise they are expanded to bf16 in ws first (exact) and the bf16 GEMM
- * runs. */
+ * MXFP4 weights: the codes are multiplied as stored on block-scaled tensor
+ * cores (tcgen05 kind::mxf8f6f4); x_perm is first quantised in ws to a hi +
+ * lo pair of E4M3 terms per element with an E8M0 scale per 32 elements each
+ * (about 8 significant bits, like bf16). Experts with 1..32 rows take a
+ * kernel with the weights on the MMA's M side, the others 128-row tiles. A
+ * block of 32 values whose largest magnitude is below 2^-119 is taken as
+ * zero; a non-finite value makes its block NaN. */
 MOE_API moe_status_t moe_mlp1(moe_dims_t d, const uint16_t* x_perm, const int32_t* offsets, moe_weight_t W1,
                       const uint16_t* b1, uint16_t* h, void* ws, size_t ws_bytes, void* stream);
 
@@ -213,8 +214,8 @@ MOE_API moe_status_t moe_forward(moe_dims_t d, const uint16_t* x, const uint16_t
  * padded with zeros -- so the GEMMs read them as contiguous runs rather than
  * as 64-byte pieces of rows K/2 bytes apart (about twice the delivered HBM
  * bandwidth on decode-sized batches). The form takes about the size of the
- * codes plus 1.5x the scales; once it exists, the original data and scales
- * are not read again. moe_mxfp4_prepare() writes the complete form for one weight
+ * codes plus 2.4x the scales (the atoms of both GEMM kernels); once it
+ * exists, the original data and scales are not read again. moe_mxfp4_prepare() writes the complete form for one weight
  * (which = 1: W1 (E, 2I, D); which = 2: W2 (E, D, I)) into `out` (device
  * memory of at least moe_mxfp4_prepared_bytes(d, which) bytes, 256-byte
  * aligned, owned by the caller), enqueued on `stream`; pass it as that

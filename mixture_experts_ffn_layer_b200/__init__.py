@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     moe_read_device_status, status_str, moe_permute_noalloc, moe_selftest_wait_timeout, mxfp4_prepared_bytes,
     moe_mxfp4_prepare, mxfp4_prepare,
 )
+from .ep import CudaLocalOps, ExpertParallelMoE, ep_forward  # noqa: F401,E402
 
 
 class MoELayer:
