@@ -91,17 +91,64 @@ def dist_env():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks, power and clock-event (throttle) reasons sampled during the
+    timed region: NVML polled from a thread every 10 ms (reads only), else
+    nvidia-smi at its 100 ms minimum period."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
+        self.thread = None
+        self.rows = []  # (sm_mhz, sm_max_mhz, power_w, reason bits)
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:  # the device torch uses, by PCI bus id (CUDA_VISIBLE_DEVICES may renumber)
+            pr = torch.cuda.get_device_properties(self.idx)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _sample(self):
+        nv, h = self.nv, self.h
+        self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), self.smax,
+                          nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(self.reasons_fn(h))))
+
+    def _poll(self):
+        import time
+
+        while not self.stop:
+            time.sleep(0.01)
+            try:
+                self._sample()
+            except Exception:
+                break
 
     def __enter__(self):
+        self.stop = False
+        try:
+            import threading
+
+            self.nv, self.h = self._nvml_handle()
+            self.smax = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            self.reasons_fn = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self._sample()  # one sample at the start, one at the end, the thread's in between
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
+            self.rows = []
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -112,6 +159,13 @@ class Clocks:
 
     def __exit__(self, *a):
         self.out = ""
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
+            try:
+                self._sample()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -121,6 +175,11 @@ class Clocks:
                 self.out, _ = self.proc.communicate()
 
     def summary(self):
+        if self.rows:
+            sm = [r[0] for r in self.rows]
+            reasons = sorted({n for r in self.rows for n, bit in self.REASONS.items() if r[3] & bit})
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(self.rows[0][1]), "reasons": reasons,
+                    "samples": len(self.rows), "power_w_max": max(r[2] for r in self.rows), "source": "nvml 10 ms"}
         rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
@@ -129,7 +188,8 @@ class Clocks:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]"))}
+                "power_w_max": max(float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]")),
+                "source": "nvidia-smi 100 ms"}
 
 
 GEMM_SOURCES = ("grouped_gemm.cu", "gemm_common.cuh", "sm100.cuh")
