@@ -733,12 +733,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // its N side, hi rows over lo rows (N = 64), one MMA per 32-K block. Each tile
 // streams its weight rows once through a deep ring of small stages, so the
 // kernel runs at the rate HBM delivers the 4.25-bit weights.
-//   warp 0      weight-side producer, per stage: the weight codes (one TMA
-//               box, 16U4_ALIGN16B, both mlp1 halves) and the weight rows'
-//               scale atom (TMA, from the preparation pass);
-//   warp 6      row-side producer, per stage: the expert's hi and lo rows (one
-//               3-D TMA box of 32 rows x 2 planes) and their 64-row scale atom
-//               (TMA, from the activation scales);
+//   warps 0, 9  weight-side producers (even / odd stages): the weight codes
+//               (one TMA box, 16U4_ALIGN16B, both mlp1 halves) and the weight
+//               rows' scale atom (TMA, from the preparation pass);
+//   warps 6, 10 row-side producers (likewise): the expert's hi and lo rows
+//               (one 3-D TMA box of 32 rows x 2 planes) and their 64-row scale
+//               atom (TMA, from the activation scales);
 //   warps 1,7,8 MMA: two scale copies into tensor memory and 4 block-scaled
 //               MMAs per stage; warp i takes the stages q = i mod 3 into its
 //               own accumulator. Each tcgen05 instruction holds its issuing
@@ -753,9 +753,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 // copies, so no proxy fence sits on the pipeline.
 constexpr int kSmallRows = 32;
 constexpr int kSN = 2 * kSmallRows;                  // the expert's hi rows, then its lo rows
-constexpr int kSThreads = 288;
 constexpr int kSIssuers = 3;
+// Producers per side. Producer i fills the stages n with n mod kSProducers =
+// i, and the ring depth is a multiple of kSProducers, so every ring slot is
+// always filled by the same thread: a producer's parity wait on a slot's
+// empty barrier is then never two phases behind (the slot's previous fill was
+// its own, issued after the phase before completed). With slots rotating
+// among producers one could run a ring ahead of another and pass a wait on
+// the stale parity.
+constexpr int kSProducers = 2;
+// warps: 0, 6 producers; 1, 7, 8 issuers; 2..5 epilogue; 9.. the other producers
+constexpr int kSThreads = 32 * (9 + 2 * (kSProducers - 1));
 __device__ __forceinline__ int small_issuer_of(int warp) { return warp == 1 ? 0 : warp == 7 ? 1 : warp == 8 ? 2 : -1; }
+// producer id: side * kSProducers + i (side 1: the row side), producer i
+// taking the stages n with n mod kSProducers = i; -1 for other warps
+static_assert(kSThreads / 32 == 9 + 2 * (kSProducers - 1), "every producer id has a warp");
+__device__ __forceinline__ int small_producer_of(int warp) {
+  if (warp == 0) return 0;
+  if (warp == 6) return kSProducers;
+  if (warp >= 9 && warp < 9 + 2 * (kSProducers - 1)) {
+    const int j = warp - 9;
+    return (j & 1) ? kSProducers + 1 + j / 2 : 1 + j / 2;
+  }
+  return -1;
+}
 constexpr uint32_t kSA = 128 * 128;                  // weight operand: 128 rows x 128 B
 constexpr uint32_t kSB = kSN * 128;                  // row operand: 64 rows x 128 B
 constexpr uint32_t kSStage = kSA + kSB + 1024;       // + weight scale atom, row scale atom (512 B each)
@@ -770,7 +791,6 @@ constexpr int kXStride = 33;                         // floats per row of the up
 __host__ __device__ constexpr uint32_t small_ctrl_bytes(int stages) {
   return (8u * static_cast<uint32_t>(3 * stages + 9) + 16u + 15u) / 16u * 16u;
 }
-constexpr int kSRowProducerWarp = 6;
 
 struct SmallParams {
   GemmParams g;           // E, K, n_out, b_rows, R, offsets, bias, perm, topk_w, out, status, act
@@ -913,14 +933,18 @@ __global__ void __launch_bounds__(kSThreads, 1)
     wt = tile - tpre[e];
   };
 
-  if (warp == 0 || warp == kSRowProducerWarp) {
+  if (small_producer_of(warp) >= 0) {
     if (lane == 0) {
       // ---------------------------------------------------------- producers
-      // (one TMA copy per operand per stage, two issuing threads: a thread
-      // waits ~60 ns after each copy it issues before the next)
-      const bool xside = warp == kSRowProducerWarp;
+      // One TMA copy per operand per stage; a thread waits ~60 ns after each
+      // copy it issues, so each side is split over kSProducers threads taking
+      // the stages in turn (each always the same ring slots: S is a multiple
+      // of kSProducers).
+      const int pid = small_producer_of(warp);
+      const bool xside = pid >= kSProducers;
+      const int par = pid % kSProducers;
       const uint32_t stage_tx = xside ? kSB + 512 : 128 * (BKE / 2) + 512;
-      int s = 0, issued = 0;
+      int s = 0, n = 0;
       uint32_t ph = 0;
       bool failed = false;
       for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
@@ -931,26 +955,28 @@ __global__ void __launch_bounds__(kSThreads, 1)
         const int wrow = kSwiGLU ? wt * 64 : wt * 128;  // the tile's first (gate) row within the expert
         const int64_t wsf_row = (static_cast<int64_t>(e) * p.NT2 + wt) * nst;
         for (int q = 0; q < nst; ++q) {
-          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
-            failed = true;
-            break;
+          if (n % kSProducers == par) {
+            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs)) {
+              failed = true;
+              break;
+            }
+            const uint32_t st = smem_u32(ring + s * kSStage);
+            const uint32_t fb = xside ? full_x(s) : full_bar(s);
+            mbar_arrive_expect_tx(fb, stage_tx);
+            if (xside) {
+              tma_load_3d(st + kSA, &tmX, fb, q * BKE, row0, 0);  // hi rows over lo rows
+              tma_load_2d(st + kSA + kSB + 512, &tmXsf, fb, 0, static_cast<int32_t>(g * nst + q));
+            } else {
+              if (p.wprep)
+                tma_load_4d(st, &tmW, fb, 0, wrow, 0, e * nst + q);
+              else if (q < nfull)
+                tma_load_4d(st, &tmW, fb, q * BKE, e * gp.b_rows + wrow, 0, 0);
+              else
+                tma_load_4d(st, &tmWtail, fb, 0, e * gp.b_rows + wrow, 0, 0);
+              tma_load_2d(st + kSA + kSB, &tmWsf, fb, 0, static_cast<int32_t>(wsf_row + q));
+            }
           }
-          const uint32_t st = smem_u32(ring + s * kSStage);
-          const uint32_t fb = xside ? full_x(s) : full_bar(s);
-          mbar_arrive_expect_tx(fb, stage_tx);
-          if (xside) {
-            tma_load_3d(st + kSA, &tmX, fb, q * BKE, row0, 0);  // hi rows over lo rows
-            tma_load_2d(st + kSA + kSB + 512, &tmXsf, fb, 0, static_cast<int32_t>(g * nst + q));
-          } else {
-            if (p.wprep)
-              tma_load_4d(st, &tmW, fb, 0, wrow, 0, e * nst + q);
-            else if (q < nfull)
-              tma_load_4d(st, &tmW, fb, q * BKE, e * gp.b_rows + wrow, 0, 0);
-            else
-              tma_load_4d(st, &tmWtail, fb, 0, e * gp.b_rows + wrow, 0, 0);
-            tma_load_2d(st + kSA + kSB, &tmWsf, fb, 0, static_cast<int32_t>(wsf_row + q));
-          }
-          ++issued;
+          ++n;
           if (++s == S) {
             s = 0;
             ph ^= 1u;
@@ -960,13 +986,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
       if (failed) {
         record_status(gp.status, MOE_ERR_TIMEOUT);
         *abort_flag = 1;
-        const int n = issued < S ? issued : S;  // this thread's copies still in flight
-        for (int i = 0; i < n; ++i) {
+        // this thread's copies still in flight: its stages among the last S
+        for (int i = 1; i <= S && i <= n; ++i) {
           if (--s < 0) {
             s = S - 1;
             ph ^= 1u;
           }
-          mbar_wait_bounded(xside ? full_x(s) : full_bar(s), ph, nullptr, kWaitNs);
+          if ((n - i) % kSProducers == par) mbar_wait_bounded(xside ? full_x(s) : full_bar(s), ph, nullptr, kWaitNs);
         }
       }
     }
@@ -988,7 +1014,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
       const uint32_t d_tmem = tmem_base + (2 * iss + acc) * kSAccStride;
       for (int q = 0; q < nst; ++q) {
         if (q % kSIssuers == iss) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs) &&
+          // The slot's previous stage may have been another issuer's: wait
+          // for it to be consumed first, so that the parity waits on the full
+          // barriers cannot match that older phase.
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, kWaitNs) &&
+                                           mbar_wait_bounded(full_bar(s), ph, abort_flag, kWaitNs) &&
                                            mbar_wait_bounded(full_x(s), ph, abort_flag, kWaitNs))) {
             failed = true;
             break;
@@ -1258,9 +1288,10 @@ template <bool kSwiGLU>
 SmallGeom small_geom(const GemmParams& g) {
   SmallGeom sg{};
   sg.NT2 = kSwiGLU ? g.n_out / 64 : (g.n_out + 127) / 128;
-  sg.stages = kSMaxStages;
-  while (sg.stages >= 3 && small_smem_bytes(sg.stages, g.E) > 227 * 1024) --sg.stages;
-  sg.ok = sg.stages >= 3 && (!kSwiGLU || g.n_out % 64 == 0);
+  // (a multiple of kSProducers: each ring slot keeps one producer)
+  sg.stages = kSMaxStages / kSProducers * kSProducers;
+  while (sg.stages >= kSProducers && small_smem_bytes(sg.stages, g.E) > 227 * 1024) sg.stages -= kSProducers;
+  sg.ok = sg.stages >= 3 && sg.stages % kSProducers == 0 && (!kSwiGLU || g.n_out % 64 == 0);
   return sg;
 }
 
