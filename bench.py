@@ -48,6 +48,7 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # kernels per step: route 1, permute 3, gather 1, mlp1 1, mlp2 1, combine 1
 LAUNCHES_PER_STEP = 8
+PERM_SINGLE_MAX = 1024  # T*k up to this: the permutation is one launch instead of three
 
 
 def act_tuple(args):
@@ -62,13 +63,14 @@ def act_config(args):
         "activation": f"gpt-oss swiglu variant (alpha {args.act_alpha}, limit {args.act_limit})"}
 
 
-def launches_per_step(T: int, D: int, mxfp4: bool) -> int:
-    """Kernel launches of one staged step: the eight above, plus for MXFP4
-    weights (prepared once) two more per GEMM -- the activation quantiser and
-    the second of the two block-scaled GEMM kernels (small-expert and
-    big-tile) -- plus the router's partial-logit reduction when it splits K
-    (batches of at most 18 token tiles of 128, D over 64)."""
-    n = LAUNCHES_PER_STEP + (4 if mxfp4 else 0)
+def launches_per_step(T: int, D: int, mxfp4: bool, k: int = 4) -> int:
+    """Kernel launches of one staged step: the eight above (the permutation
+    in one launch instead of three when T*k <= PERM_SINGLE_MAX), plus for
+    MXFP4 weights (prepared once) two more per GEMM -- the activation
+    quantiser and the second of the two block-scaled GEMM kernels
+    (small-expert and big-tile) -- plus the router's partial-logit reduction
+    when it splits K (batches of at most 18 token tiles of 128, D over 64)."""
+    n = LAUNCHES_PER_STEP + (4 if mxfp4 else 0) - (2 if T * k <= PERM_SINGLE_MAX else 0)
     tiles, kb = -(-T // 128), -(-D // 64)
     if tiles * 8 <= 148 and min(kb, 148 // tiles) > 1:
         n += 1
@@ -489,7 +491,7 @@ def run_ours(args):
                            "their own streams, double-buffered, overlapping neighbouring steps' compute"},
             "e2e_serial": {"value": T * world / (e2e_serial_ms / args.steps / 1e3), "unit": UNIT,
                            "how": "same, copy-compute-copy serialised on one stream"},
-            "gpu_launches": launches_per_step(T, D, mx) * args.steps,
+            "gpu_launches": launches_per_step(T, D, mx, k) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

@@ -72,45 +72,17 @@ __global__ void __launch_bounds__(kPermThreads) perm_scan_kernel(int32_t* __rest
   if (tid == 0) counts[e] = carry;
 }
 
-__global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
-                                                                    int chunk, const int32_t* __restrict__ block_pre,
-                                                                    const int32_t* __restrict__ counts,
-                                                                    int32_t* __restrict__ offsets,
-                                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+// Stable ranking of the assignments [a0, a0 + n) into perm / inv, in order,
+// kPermThreads at a time: base[e] (shared) holds the next position for expert
+// e and advances past each group; wcnt is per-warp scratch. Warp match/popc
+// and per-warp counts fix each position from (expert, a), never by atomics.
+// Every thread of the block calls it.
+__device__ void rank_assignments(const int32_t* __restrict__ idx, int64_t R, int E, int64_t a0, int n, int* base,
+                                 int (*wcnt)[256], int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   constexpr int kWarps = kPermThreads / 32;
-  __shared__ int base[256];
-  __shared__ int wcnt[kWarps][256];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int blk = blockIdx.x;
-
-  // Expert offsets (exclusive scan of the totals over experts, E <= 256 =
-  // the block size) plus this block's prefix over the blocks before it.
-  {
-    const int c = tid < E ? counts[tid] : 0;
-    int incl = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += u;
-    }
-    if (lane == 31) wcnt[0][warp] = incl;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += wcnt[0][w];
-    const int off = before + incl - c;
-    if (tid < E) {
-      base[tid] = off + block_pre[static_cast<int64_t>(blk) * E + tid];
-      if (blk == 0) {
-        offsets[tid] = off;
-        if (tid == E - 1) offsets[E] = off + c;
-      }
-    }
-    __syncthreads();
-  }
-
-  const int64_t a0 = static_cast<int64_t>(blk) * chunk;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int sub = 0; sub < chunk; sub += kPermThreads) {
+  for (int sub = 0; sub < n; sub += kPermThreads) {
     for (int i = tid; i < kWarps * 256; i += kPermThreads) (&wcnt[0][0])[i] = 0;
     __syncthreads();
     const int64_t a = a0 + sub + tid;
@@ -139,6 +111,86 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_
     __syncthreads();
     if (a0 + sub + kPermThreads >= R) break;
   }
+}
+
+// Exclusive scan of c (one value per thread, E <= 256 = the block size) over
+// the experts: returns thread tid's prefix. scratch: kPermThreads / 32 ints.
+__device__ int expert_prefix(int c, int* scratch) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  int incl = c;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += scratch[w];
+  __syncthreads();
+  return before + incl - c;
+}
+
+__global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
+                                                                    int chunk, const int32_t* __restrict__ block_pre,
+                                                                    const int32_t* __restrict__ counts,
+                                                                    int32_t* __restrict__ offsets,
+                                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  constexpr int kWarps = kPermThreads / 32;
+  __shared__ int base[256];
+  __shared__ int wcnt[kWarps][256];
+  const int tid = threadIdx.x;
+  const int blk = blockIdx.x;
+  // Expert offsets (exclusive scan of the totals over experts) plus this
+  // block's prefix over the blocks before it.
+  const int c = tid < E ? counts[tid] : 0;
+  const int off = expert_prefix(c, &wcnt[0][0]);
+  if (tid < E) {
+    base[tid] = off + block_pre[static_cast<int64_t>(blk) * E + tid];
+    if (blk == 0) {
+      offsets[tid] = off;
+      if (tid == E - 1) offsets[E] = off + c;
+    }
+  }
+  __syncthreads();
+  rank_assignments(idx, R, E, static_cast<int64_t>(blk) * chunk, chunk, base, wcnt, perm, inv);
+}
+
+// The whole permutation in one block, for batches of at most kPermSingleMax
+// assignments (decode-sized): histogram in shared memory, counts and offsets,
+// then the same stable ranking over all R assignments -- one launch instead
+// of three, the same perm / inv / counts / offsets.
+constexpr int kPermSingleMax = 1024;
+
+__global__ void __launch_bounds__(kPermThreads) perm_single_kernel(const int32_t* __restrict__ idx, int64_t R, int E,
+                                                                   int32_t* __restrict__ counts,
+                                                                   int32_t* __restrict__ offsets,
+                                                                   int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                   int* status) {
+  constexpr int kWarps = kPermThreads / 32;
+  __shared__ int base[256];
+  __shared__ int wcnt[kWarps][256];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 256; e += kPermThreads) base[e] = 0;
+  __syncthreads();
+  for (int64_t a = tid; a < R; a += kPermThreads) {
+    const int e = idx[a];
+    if (e >= 0 && e < E)
+      atomicAdd(&base[e], 1);
+    else
+      record_status(status, MOE_ERR_DEVICE_BOUNDS);
+  }
+  __syncthreads();
+  const int c = tid < E ? base[tid] : 0;
+  const int off = expert_prefix(c, &wcnt[0][0]);
+  if (tid < E) {
+    counts[tid] = c;
+    offsets[tid] = off;
+    if (tid == E - 1) offsets[E] = off + c;
+    base[tid] = off;
+  }
+  __syncthreads();
+  rank_assignments(idx, R, E, 0, static_cast<int>(R), base, wcnt, perm, inv);
 }
 
 // x_perm[r, :] = x[perm[r] / k, :]. Grid (row, chunk block): each thread
@@ -204,6 +256,10 @@ cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t
                            int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
                            int chunk) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
+  if (R <= kPermSingleMax) {
+    perm_single_kernel<<<1, kPermThreads, 0, s>>>(topk_idx, R, d.E, counts, offsets, perm, inv, status);
+    return cudaGetLastError();
+  }
   const int nblk = static_cast<int>((R + chunk - 1) / chunk);
   perm_hist_kernel<<<nblk, kPermThreads, 0, s>>>(topk_idx, R, d.E, chunk, block_counts, status);
   perm_scan_kernel<<<d.E, kPermThreads, 0, s>>>(block_counts, nblk, d.E, counts);
