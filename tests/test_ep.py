@@ -146,3 +146,18 @@ def test_blocks_pair_every_send_with_a_receive():
     for r in range(world):
         out_runs, _ = runs[r]
         assert sum(n for *_, n in out_runs) == sum(counts[r])
+
+
+def test_ep_refuses_experts_that_do_not_shard_evenly(monkeypatch):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        inp = synthetic.make_custom(4, 64, 3, 1, 64, seed=1, device="cpu")
+        ops = OracleOps(inp, 0, 1, 1)
+        y = ep.ep_forward(inp.x, ops, 3)  # one rank holds all three experts
+        assert y.shape == (4, 64)
+        # two ranks cannot hold three experts evenly: refused before any exchange
+        monkeypatch.setattr(ep, "_group_info", lambda group: (2, 0))
+        with pytest.raises(ValueError):
+            ep.ep_forward(inp.x, ops, 3)
+    finally:
+        dist.destroy_process_group()

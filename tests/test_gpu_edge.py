@@ -299,3 +299,47 @@ def test_random_shapes(T, D, E, k, I, wfmt):
     # streamed, the router with or without its K split -- against the oracle
     inp = synthetic.make_custom(T, D, E, k, I, seed=T * 7 + E, device="cuda", wfmt=wfmt, reject=oracle.gap_reject())
     _check_full(inp, TOL_MXFP4 if wfmt == "mxfp4" else TOL_BF16)
+
+
+@pytest.mark.parametrize("T,k,E", [
+    (256, 4, 32),    # T*k = 1024: the whole permutation in one block
+    (205, 5, 64),    # 1025: the three-launch path
+    (128, 8, 256),   # 1024 at the largest E and k
+    (1, 1, 1),       # one assignment
+])
+def test_permutation_on_both_sides_of_the_one_block_limit(T, k, E):
+    # the one-block and the multi-block permutation give the oracle's stable
+    # counting sort exactly (torchtitan GPT-OSS guide, "grouped matrix
+    # multiplication": counts, offsets = cumsum), with and without a workspace
+    g = torch.Generator().manual_seed(T * 31 + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    counts, offsets, perm, inv = oracle.permute(idx, E)
+    d = moe.dims(T, 64, E, k, 64)
+    ws = moe.alloc_workspace(d)
+    i32 = dict(dtype=torch.int32, device="cuda")
+    for noalloc in (False, True):
+        out = [torch.full((E,), -7, **i32), torch.full((E + 1,), -7, **i32), torch.full((T * k,), -7, **i32),
+               torch.full((T * k,), -7, **i32)]
+        if noalloc:
+            moe.moe_permute_noalloc(d, idx.cuda(), *out)
+        else:
+            moe.moe_permute(d, idx.cuda(), *out, ws)
+            assert moe.moe_read_device_status(ws) == 0
+        for a, b in zip(out, (counts, offsets, perm, inv)):
+            assert torch.equal(a.cpu(), b)
+
+
+def test_one_block_permutation_reports_out_of_range_indices():
+    T, E, k = 100, 8, 2  # T*k = 200: the one-block path
+    d = moe.dims(T, 64, E, k, 64)
+    ws = moe.alloc_workspace(d)
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32, device="cuda")
+    idx[5, 1] = E
+    idx[77, 0] = -3
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    perm, inv = torch.empty(T * k, **i32), torch.empty(T * k, **i32)
+    moe.moe_permute(d, idx, counts, offsets, perm, inv, ws)
+    assert moe.moe_read_device_status(ws) == 6
+    assert int(inv[5 * k + 1]) == -1 and int(inv[77 * k]) == -1
+    assert int(offsets[-1]) == T * k - 2 and int(counts.sum()) == T * k - 2
