@@ -74,10 +74,8 @@ cudaError_t launch_route(const moe_dims_t& d, const uint16_t* x, const uint16_t*
 cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* block_counts, int* status, cudaStream_t s,
                            int chunk = kPermChunk);
-// to_f16: write the gathered rows as f16 (the MXFP4 weight-streaming kernels'
-// input form) instead of bf16.
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm,
-                          int* status, cudaStream_t s, bool to_f16 = false);
+                          int* status, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims_t& d, const float* o_perm, const int32_t* inv, uint16_t* y,
                            int* status, cudaStream_t s);
 

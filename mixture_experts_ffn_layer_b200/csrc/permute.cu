@@ -194,9 +194,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_single_kernel(const int32_t
 }
 
 // x_perm[r, :] = x[perm[r] / k, :]. Grid (row, chunk block): each thread
-// copies one 32-byte vector (16 bf16) of one row; kF16 stores them as f16
-// (round to nearest) instead.
-template <bool kF16>
+// copies one 32-byte vector (16 bf16) of one row.
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
                                    uint16_t* __restrict__ x_perm, int64_t R, int k, int D, int* status) {
   const int64_t r = blockIdx.x;
@@ -208,13 +206,6 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
     sm100::ld_global_v8u(x + static_cast<int64_t>(a / k) * D + 16 * c, v);
   else if (c == 0)
     record_status(status, MOE_ERR_DEVICE_BOUNDS);
-  if (kF16) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float lo = __uint_as_float(v[q] << 16), hi = __uint_as_float(v[q] & 0xffff0000u);
-      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v[q]) : "f"(hi), "f"(lo));
-    }
-  }
   sm100::st_global_v8u(x_perm + r * D + 16 * c, v);
 }
 
@@ -269,14 +260,11 @@ cudaError_t launch_permute(const moe_dims_t& d, const int32_t* topk_idx, int32_t
 }
 
 cudaError_t launch_gather(const moe_dims_t& d, const uint16_t* x, const int32_t* perm, uint16_t* x_perm, int* status,
-                          cudaStream_t s, bool to_f16) {
+                          cudaStream_t s) {
   const int64_t R = static_cast<int64_t>(d.T) * d.k;
   const int n = d.D / 16, bs = row_block(n);
   const dim3 grid(static_cast<unsigned>(R), (n + bs - 1) / bs);
-  if (to_f16)
-    gather_rows_kernel<true><<<grid, bs, 0, s>>>(x, perm, x_perm, R, d.k, d.D, status);
-  else
-    gather_rows_kernel<false><<<grid, bs, 0, s>>>(x, perm, x_perm, R, d.k, d.D, status);
+  gather_rows_kernel<<<grid, bs, 0, s>>>(x, perm, x_perm, R, d.k, d.D, status);
   return cudaGetLastError();
 }
 

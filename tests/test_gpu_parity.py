@@ -102,8 +102,8 @@ def test_full_size_sampled(name):
 
 @pytest.mark.parametrize("T", [64, 8, 1024])
 def test_mxfp4_layer(T):
-    # T = 64 and 8 take the weight-streaming path (<= 16 rows per expert on
-    # average); T = 1024 expands the weights to bf16 and runs the tcgen05 GEMMs
+    # T = 64 and 8: every expert has at most 32 rows (the small-expert
+    # block-scaled kernel); T = 1024: 128-row tiles (the big-tile kernel)
     inp = _inputs("gptoss20b_mxfp4_decode", T=T)
     run = run_stages(inp)
     assert run.status == 0
