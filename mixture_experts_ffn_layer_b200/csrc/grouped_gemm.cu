@@ -39,6 +39,10 @@ using namespace sm100;
 constexpr int BM = 128;               // rows per tile = TMEM lanes
 constexpr int BK = 64;                // K per stage: one 128-byte swizzle row of bf16
 constexpr int kStages = 4;
+// Experts with at most this many rows (one m-tile) get HBM-bound tiles: each
+// column tile streams its weight slab for few rows. (Counting two-m-tile
+// experts in as well measured slower on the skewed 120B shape.)
+constexpr int kLightRows = BM;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer
@@ -60,7 +64,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
   int* bad_s = reinterpret_cast<int*>(tmem_slot + 3);
   int* seg = reinterpret_cast<int*>(ctrl + kCtrlBytes);  // E+1 segment starts
-  int* tpre = seg + (p.E + 1);                           // E+1 tile prefix
+  int* tpre = seg + (p.E + 1);                           // E+1 tile prefix, experts with > kLightRows rows
+  int* tpre1 = tpre + (p.E + 1);                         // E+1 tile prefix, experts with 1..kLightRows rows
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t bar0 = smem_u32(bars);
@@ -86,30 +91,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile counts per expert, exclusive scan across the warp (E <= 256)
     const int per = (p.E + 31) / 32;
     const int e0 = lane * per;
-    int local = 0;
+    // two tile lists: experts with more than kLightRows rows (tensor-bound)
+    // and experts with 1..kLightRows rows (HBM-bound)
+    int local = 0, local1 = 0;
     for (int e = e0; e < e0 + per && e < p.E; ++e) {
       const int cnt = seg[e + 1] - seg[e];
       if (cnt < 0) atomicOr(bad_s, 1);
-      local += cnt > 0 ? (cnt + BM - 1) / BM * p.NT : 0;
+      if (cnt > kLightRows)
+        local += (cnt + BM - 1) / BM * p.NT;
+      else if (cnt > 0)
+        local1 += (cnt + BM - 1) / BM * p.NT;
     }
-    int incl = local;
+    int incl = local, incl1 = local1;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
+      const int v = __shfl_up_sync(0xffffffffu, incl, off), v1 = __shfl_up_sync(0xffffffffu, incl1, off);
+      if (lane >= off) {
+        incl += v;
+        incl1 += v1;
+      }
     }
-    int run = incl - local;
+    int run = incl - local, run1 = incl1 - local1;
     for (int e = e0; e < e0 + per && e < p.E; ++e) {
       tpre[e] = run;
+      tpre1[e] = run1;
       const int cnt = seg[e + 1] - seg[e];
-      run += cnt > 0 ? (cnt + BM - 1) / BM * p.NT : 0;
+      if (cnt > kLightRows)
+        run += (cnt + BM - 1) / BM * p.NT;
+      else if (cnt > 0)
+        run1 += (cnt + BM - 1) / BM * p.NT;
     }
-    if (lane == 31) tpre[p.E] = incl;
+    if (lane == 31) {
+      tpre[p.E] = incl;
+      tpre1[p.E] = incl1;
+    }
     __syncwarp();
     if (lane == 0) {
       const int bad = *bad_s;
       if (bad) record_status(p.status, MOE_ERR_DEVICE_BOUNDS);
-      *total_s = bad ? 0 : tpre[p.E];
+      *total_s = bad ? 0 : tpre[p.E] + tpre1[p.E];
       for (int s = 0; s < kStages; ++s) {
         mbar_init(full_bar(s), 1);
         mbar_init(empty_bar(s), 1);
@@ -133,6 +153,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = *total_s;
   const int KB = (p.K + BK - 1) / BK;
+  // Schedule position -> tile. The light experts' tiles are spread
+  // evenly among the others (position i takes the next one of them when
+  // floor((i+1) C / total) steps, C their number), so that every wave of
+  // concurrent tiles mixes HBM-bound and tensor-bound work; each list keeps
+  // its own order (consecutive tiles of an expert share its weights in L2).
+  const int n_single = tpre1[p.E];
+  auto schedule = [&](int i, int& e, int& nt, int& mt) {
+    const int64_t c0 = static_cast<int64_t>(i) * n_single / total;
+    const int64_t c1 = static_cast<int64_t>(i + 1) * n_single / total;
+    if (c1 > c0)
+      decode_tile(static_cast<int>(c0), tpre1, seg, p.E, BM, e, nt, mt);
+    else
+      decode_tile(i - static_cast<int>(c0), tpre, seg, p.E, BM, e, nt, mt);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -143,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool failed = false;
       for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
         int e, nt, mt;
-        decode_tile(tile, tpre, seg, p.E, BM, e, nt, mt);
+        schedule(tile, e, nt, mt);
         const int row0 = seg[e] + mt * BM;
         const int brow = e * p.b_rows + nt * p.n_tile;
         for (int kb = 0; kb < KB; ++kb) {
@@ -238,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int e, nt, mt;
-      decode_tile(tile, tpre, seg, p.E, BM, e, nt, mt);
+      schedule(tile, e, nt, mt);
       const bool ok = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag, kWaitNs);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) {
@@ -278,7 +312,7 @@ int pick_tile(int n, int max_tile, int step) {
 }
 
 size_t smem_bytes(int mma_n, int E) {
-  return 1024 + static_cast<size_t>(kStages) * (kABytes + mma_n * BK * 2) + kCtrlBytes + 2 * (E + 1) * sizeof(int);
+  return 1024 + static_cast<size_t>(kStages) * (kABytes + mma_n * BK * 2) + kCtrlBytes + 3 * (E + 1) * sizeof(int);
 }
 
 template <bool kSwiGLU>
