@@ -731,8 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // weights are the MMA's M side, 128 weight rows per tile (mlp1: 64 gate rows
 // over the 64 matching up rows; mlp2: 128 output rows), and the expert's rows
 // its N side, hi rows over lo rows (N = 64), one MMA per 32-K block. Each tile
-// streams its weight rows once through a deep ring of small stages, so the
-// kernel runs at the rate HBM delivers the 4.25-bit weights.
+// streams its weight rows once through a deep ring of small stages: every
+// weight byte crosses HBM once, at 4.25 bits per element.
 //   warps 0, 9  weight-side producers (even / odd stages): the weight codes
 //               (one TMA box, 16U4_ALIGN16B, both mlp1 halves) and the weight
 //               rows' scale atom (TMA, from the preparation pass);
@@ -742,15 +742,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warps 1,7,8 MMA: two scale copies into tensor memory and 4 block-scaled
 //               MMAs per stage; warp i takes the stages q = i mod 3 into its
 //               own accumulator. Each tcgen05 instruction holds its issuing
-//               warp for ~50 ns, so one warp needs ~0.4 us per stage where HBM
-//               delivers one in ~0.2; issuing from three warps overlaps it;
+//               warp for ~50 ns (~0.4 us for a stage's seven), so the stages
+//               are spread over three issuing warps;
 //   warps 2..5  epilogue (lane = weight row): the issuers' hi + lo parts
 //               added per row in a fixed order, then SwiGLU with the up half
 //               from the other two warps via shared memory and h quantised
 //               across the warp's 32 columns, or bias * gate weight into the
 //               fp32 expert outputs.
-// Nothing here writes shared memory for the tensor core but TMA and the bulk
-// copies, so no proxy fence sits on the pipeline.
+// Nothing here writes shared memory for the tensor core but TMA, so no proxy
+// fence sits on the pipeline.
 constexpr int kSmallRows = 32;
 constexpr int kSN = 2 * kSmallRows;                  // the expert's hi rows, then its lo rows
 constexpr int kSIssuers = 3;
